@@ -1,0 +1,58 @@
+"""The seeded input generators: deterministic, sliceable, and of the stated
+distributions and routing structure."""
+
+import numpy as np
+import torch
+
+from fp8_fine_grained_permute_b200 import workloads as W
+
+
+def test_slices_regenerate_identically():
+    cfg = W.CONFIGS["kanana"]
+    full = W.gen_normal_bf16((4, 1536, 256), 0.02, cfg.seed, W.SID_W_UP)
+    part = W.gen_normal_bf16((1536, 256), 0.02, cfg.seed, W.SID_W_UP, index_offset=2 * 1536 * 256)
+    assert torch.equal(full[2].view(torch.int16), part.view(torch.int16))
+    idx = torch.tensor([5, 1536 * 256 * 3 + 7], dtype=torch.int64)
+    at = W.gen_normal_bf16_at(idx, 0.02, cfg.seed, W.SID_W_UP)
+    assert at[0].item() == full.view(-1)[5].item() and at[1].item() == full.view(-1)[idx[1]].item()
+
+
+def test_streams_differ_and_repeat():
+    a = W.gen_normal_bf16((1000,), 1.0, 1, 1)
+    b = W.gen_normal_bf16((1000,), 1.0, 1, 2)
+    c = W.gen_normal_bf16((1000,), 1.0, 1, 1)
+    assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+    assert not torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_large_index_streams():
+    # indices beyond 2^32 (the largest weight tensors have ~7.5e9 elements)
+    lo = W.gen_normal_bf16((64,), 1.0, 3, 3, index_offset=5)
+    hi = W.gen_normal_bf16((64,), 1.0, 3, 3, index_offset=5 + (1 << 32))
+    assert not torch.equal(lo.view(torch.int16), hi.view(torch.int16))
+
+
+def test_distributions():
+    x = W.gen_normal_bf16((1 << 20,), 1.0, 9, 1).float()
+    assert abs(x.mean().item()) < 5e-3 and abs(x.std().item() - 1.0) < 5e-3
+    w = W.gen_normal_bf16((1 << 20,), 0.02, 9, 2).float()
+    assert abs(w.std().item() - 0.02) < 2e-4
+    g = W.gen_grad_bf16((1 << 20,), 9, 5).float()
+    # 0.1 % of entries are x100: P(|t3| > 0.5) = 0.65, so ~6.5e-4 of entries exceed 50
+    # (the plain t3 tail above 50 adds ~1.6e-5)
+    big = (g.abs() > 50).float().mean().item()
+    assert 5e-4 < big < 8.5e-4
+    med = g.abs().median().item()
+    assert abs(med - 0.765) < 0.02                           # median |t_3| = 0.7649
+
+
+def test_routing_structure():
+    for name in ("tiny", "kanana", "dsv3"):
+        cfg = W.CONFIGS[name]
+        ids = W.route(cfg)
+        assert ids.shape == (cfg.T, cfg.k) and ids.dtype == np.int32
+        assert ids.min() >= 0 and ids.max() < cfg.E
+        assert all(len(set(r)) == cfg.k for r in ids)       # distinct experts per token
+        assert np.array_equal(ids, W.route(cfg))             # deterministic
+    counts = np.bincount(W.route(W.CONFIGS["dsv3"]).ravel(), minlength=256)
+    assert (counts == 0).sum() == 16 and counts.max() > 4000  # Zipf skew + forced empties
