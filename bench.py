@@ -1,0 +1,557 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 fine-grained MoE path on B200.
+
+One step = one pass of the whole path over one batch of the DeepSeek-V3-shaped
+MoE layer (256 experts, hidden 7168, inter 2048, 8192 tokens top-8, Zipf(1.2)
+routing with 16 empty experts), forward and backward shapes:
+
+  K1  permute + 1x128 quantize X [8192, 7168]            (fg8_quantize_act, rowwise)
+  K2  128x128 quantize W_up [256, 4096, 7168], W_down [256, 7168, 2048]
+  K4  fprop up    Y_up   = Xq  . Wq_up^T     -> bf16 [65536, 4096]
+  K1  1x128 quantize H [65536, 2048] (down-projection input, in expert order)
+  K4  fprop down  Y_down = Hq  . Wq_down^T   -> bf16 [65536, 7168]
+  K3  transpose Wq_up -> WqT_up [256, 7168, 4096] (+ scale grid)
+  K1  1x128 quantize dY [65536, 4096]
+  K4  dgrad       dX     = dYq . WqT_up^T    -> bf16 [65536, 7168]
+  K1  column-wise quantize dY and X (gathered by row) along tokens, per expert
+  K4  wgrad       dW_e   = dY_e^T X_e        -> fp32 [256, 4096, 7168]
+
+The printed `value` is the grouped FP8 GEMM throughput (algorithmic FLOPs of
+the four GEMMs over their summed kernel time, CUDA events on the launching
+stream); `quantize_gbs` is the same for the bandwidth kernels.  `roofline`
+describes the kernel with the largest share of the step; `kernels` lists
+every kernel against its own roofline.
+
+`--impl reference` times the CPU oracle (the reference implementation of what
+the path computes) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp8_fine_grained_permute_b200 import workloads as W  # noqa: E402
+
+METRIC = "grouped FP8 GEMM TFLOP/s + quantize GB/s, % of B200 FP8/HBM roofline"
+FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=FALLBACK["hbm_gbs"], bf16=FALLBACK["bf16_tflops"],
+                bf16_sus=FALLBACK["bf16_tflops_sustained"], source="fallback")
+
+
+# --------------------------------------------------------------------------
+# algorithmic work per kernel launch (bytes the method must move, FLOPs it must do)
+# --------------------------------------------------------------------------
+
+def bytes_route_quant(T, K, k, E):
+    R = T * k
+    return 2 * T * K + R * K + 4 * R * K // 128 + 4 * T * k + 8 * R + 4 * (E + 1)
+
+
+def bytes_rows_quant(R, K):
+    return 2 * R * K + R * K + 4 * R * K // 128
+
+
+def bytes_colwise(read_rows, C, padded_total):
+    return 2 * read_rows * C + padded_total * C + 4 * padded_total * C // 128
+
+
+def bytes_weight_quant(E, N, K):
+    return 3 * E * N * K + 4 * E * N * K // 16384
+
+
+def bytes_transpose(E, N, K):
+    return 2 * (E * N * K + 4 * E * N * K // 16384)
+
+
+# --------------------------------------------------------------------------
+# the workload on one GPU
+# --------------------------------------------------------------------------
+
+class Step:
+    """Device-resident inputs and outputs of one step; `run` launches the path."""
+
+    def __init__(self, cfg: W.MoEConfig, dev):
+        from fp8_fine_grained_permute_b200 import fg8
+        self.fg8 = fg8
+        self.cfg = cfg
+        self.dev = dev
+        T, K, k, E, R = cfg.T, cfg.hidden, cfg.k, cfg.E, cfg.R
+        N, I = cfg.n_up, cfg.inter
+        self.ids_np = W.route(cfg)
+        counts = np.bincount(self.ids_np.ravel(), minlength=E)
+        self.padded_total = int(((counts + 127) // 128 * 128).sum())
+        u8, f32, i32, bf = torch.uint8, torch.float32, torch.int32, torch.bfloat16
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)  # noqa: E731
+        # inputs (generated on the device by the seeded counter-based generators)
+        self.x = W.gen_x(cfg, dev)
+        self.ids = torch.from_numpy(self.ids_np).to(dev)
+        self.w_up = W.gen_w_up(cfg, dev)
+        self.w_down = W.gen_w_down(cfg, dev) if I else None
+        self.h = W.gen_h(cfg, dev) if I else None
+        self.dy = W.gen_dy(cfg, dev)
+        # outputs / intermediates
+        self.xq, self.sa = e((R, K), u8), e((K // 128, R), f32)
+        self.row_token, self.token_row = e(R, i32), e(T * k, i32)
+        self.offsets = e(E + 1, i32)
+        self.ws_bytes = fg8.fg8_quantize_act_workspace(T, k, E)
+        self.ws = e(self.ws_bytes, u8)
+        self.status = torch.zeros(1, dtype=i32, device=dev)
+        self.wq_up, self.sw_up = e((E, N, K), u8), e((E, N // 128, K // 128), f32)
+        self.y_up = e((R, N), bf)
+        if I:
+            self.wq_dn, self.sw_dn = e((E, K, I), u8), e((E, K // 128, I // 128), f32)
+            self.hq, self.sh = e((R, I), u8), e((I // 128, R), f32)
+            self.y_dn = e((R, K), bf)
+        self.wqT_up, self.swT_up = e((E, K, N), u8), e((E, K // 128, N // 128), f32)
+        self.dyq, self.sdy = e((R, N), u8), e((N // 128, R), f32)
+        self.dx = e((R, K), bf)
+        self.P = fg8.fg8_colwise_capacity(R, E)
+        self.dyT, self.sdyT, self.pad_dy = e((N, self.P), u8), e((self.P // 128, N), f32), e(E + 1, i32)
+        self.xT, self.sxT, self.pad_x = e((K, self.P), u8), e((self.P // 128, K), f32), e(E + 1, i32)
+        self.dw = e((E, N, K), f32)
+        self.launches_per_step = 0
+        self.work = self._work()
+
+    def _work(self):
+        c = self.cfg
+        T, K, k, E, R, N, I = c.T, c.hidden, c.k, c.E, c.R, c.n_up, c.inter
+        w = {
+            "quant_act_permute": ("hbm", bytes_route_quant(T, K, k, E)),
+            "quant_weight": ("hbm", bytes_weight_quant(E, N, K) + (bytes_weight_quant(E, K, I) if I else 0)),
+            "gemm_fprop_up": ("tensor", 2 * R * N * K),
+            "transpose_blockq": ("hbm", bytes_transpose(E, N, K)),
+            "quant_act_rows": ("hbm", bytes_rows_quant(R, N) + (bytes_rows_quant(R, I) if I else 0)),
+            "gemm_dgrad": ("tensor", 2 * R * K * N),
+            "quant_act_colwise": ("hbm", bytes_colwise(R, N, self.padded_total) +
+                                  bytes_colwise(T, K, self.padded_total)),
+            "gemm_wgrad": ("tensor", 2 * R * N * K),
+        }
+        if I:
+            w["gemm_fprop_down"] = ("tensor", 2 * R * K * I)
+        return w
+
+    def run(self, stream, marks=None):
+        """Launch one step on `stream`.  With `marks`, record an event pair
+        around each kernel family: marks[name] -> list of (start, end)."""
+        fg8, c = self.fg8, self.cfg
+        T, K, k, E, R, N, I = c.T, c.hidden, c.k, c.E, c.R, c.n_up, c.inter
+        sp = stream.cuda_stream
+        n = [0]
+
+        def timed(name, fn):
+            if marks is not None:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                marks.setdefault(name, []).append((a, b))
+            else:
+                fn()
+
+        def launch(fn):
+            def g():
+                fn()
+                n[0] += 1
+            return g
+
+        u16 = lambda t: t.view(torch.int16)  # noqa: E731
+        timed("quant_act_permute", launch(lambda: fg8.fg8_quantize_act(
+            u16(self.x), T, K, self.ids, k, E, None, fg8.FG8_ROWWISE, self.xq, self.sa,
+            self.row_token, self.token_row, self.offsets, None, None, self.ws, self.ws_bytes,
+            self.status, sp)))
+
+        def wquant():
+            fg8.fg8_quantize_weight(u16(self.w_up), E, N, K, self.wq_up, self.sw_up, sp)
+            n[0] += 1
+            if I:
+                fg8.fg8_quantize_weight(u16(self.w_down), E, K, I, self.wq_dn, self.sw_dn, sp)
+                n[0] += 1
+        timed("quant_weight", wquant)
+        timed("gemm_fprop_up", launch(lambda: fg8.fg8_grouped_gemm(
+            self.xq, self.sa, self.wq_up, self.sw_up, self.offsets, R, N, K, E, fg8.FG8_GROUP_M,
+            fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_up, self.status, sp)))
+
+        def rows():
+            if I:
+                fg8.fg8_quantize_act(u16(self.h), R, I, None, 1, 1, None, fg8.FG8_ROWWISE, self.hq,
+                                     self.sh, None, None, None, None, None, None, 0, None, sp)
+                n[0] += 1
+            fg8.fg8_quantize_act(u16(self.dy), R, N, None, 1, 1, None, fg8.FG8_ROWWISE, self.dyq,
+                                 self.sdy, None, None, None, None, None, None, 0, None, sp)
+            n[0] += 1
+        timed("quant_act_rows", rows)
+        if I:
+            timed("gemm_fprop_down", launch(lambda: fg8.fg8_grouped_gemm(
+                self.hq, self.sh, self.wq_dn, self.sw_dn, self.offsets, R, K, I, E,
+                fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_dn,
+                self.status, sp)))
+        timed("transpose_blockq", launch(lambda: fg8.fg8_transpose_blockq(
+            self.wq_up, self.sw_up, E, N, K, self.wqT_up, self.swT_up, sp)))
+        timed("gemm_dgrad", launch(lambda: fg8.fg8_grouped_gemm(
+            self.dyq, self.sdy, self.wqT_up, self.swT_up, self.offsets, R, K, N, E,
+            fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.dx, self.status, sp)))
+
+        def colwise():
+            fg8.fg8_quantize_act(u16(self.dy), R, N, None, 1, E, self.offsets, fg8.FG8_COLWISE,
+                                 None, None, None, None, self.pad_dy, self.dyT, self.sdyT, None, 0,
+                                 None, sp)
+            fg8.fg8_quantize_act(u16(self.x), T, K, None, k, E, self.offsets, fg8.FG8_COLWISE,
+                                 None, None, self.row_token, None, self.pad_x, self.xT, self.sxT,
+                                 None, 0, None, sp)
+            n[0] += 2
+        timed("quant_act_colwise", colwise)
+        timed("gemm_wgrad", launch(lambda: fg8.fg8_grouped_gemm(
+            self.dyT, self.sdyT, self.xT, self.sxT, self.pad_dy, N, K, self.P, E, fg8.FG8_GROUP_K,
+            fg8.FG8_BSCALE_ROW128, fg8.FG8_OUT_F32, self.dw, self.status, sp)))
+        self.launches_per_step = n[0]
+
+    # host-side inputs / outputs of the end-to-end measurement
+    def host_io(self):
+        pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+        ins = [(pin(self.x), self.x), (pin(self.ids), self.ids), (pin(self.dy), self.dy)]
+        if self.h is not None:
+            ins.append((pin(self.h), self.h))
+        res = self.y_dn if self.h is not None else self.y_up
+        outs = [(torch.empty(res.shape, dtype=res.dtype).pin_memory(), res),
+                (torch.empty(self.dx.shape, dtype=self.dx.dtype).pin_memory(), self.dx)]
+        return ins, outs
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# --------------------------------------------------------------------------
+
+class OracleSample:
+    """The oracle, as it stands, on a bounded sample of the workload: permute +
+    1x128 quantize of the first tokens, 128x128 quantize and transpose of a
+    slab of one expert's up-projection weight, and the fp64 GEMM of whole
+    output rows against that expert.  Inputs are generated once, outside the
+    timed calls."""
+
+    def __init__(self, cfg: W.MoEConfig, ntok: int = 32, wrows: int = 512):
+        import oracle
+        oracle.build()
+        self.o = oracle
+        self.cfg = cfg
+        K, N, E = cfg.hidden, cfg.n_up, cfg.E
+        ids = W.route(cfg)
+        counts = np.bincount(ids.ravel(), minlength=E)
+        self.e = int(np.argmax(counts))
+        self.ntok = ntok
+        self.ids = np.ascontiguousarray(ids[:ntok])
+        self.x = W.gen_x(cfg)[:ntok].contiguous()
+        self.wrows = min(wrows, N)
+        self.w = W.gen_w_up(cfg, experts=[self.e])[:, :self.wrows].contiguous()
+        act = oracle.quantize_act(self.x[:8].contiguous(), None, 1)
+        self.a_rows, self.sa_rows = act["xq"], act["sa"]
+        self.q_bytes = (bytes_route_quant(ntok, K, cfg.k, E) + bytes_weight_quant(1, self.wrows, K) +
+                        bytes_transpose(1, self.wrows, K))
+
+    def run(self, gemm_budget_s: float):
+        o, K = self.o, self.cfg.hidden
+        t0 = time.perf_counter()
+        o.quantize_act(self.x, self.ids, self.cfg.E)
+        wq, sw = o.quantize_weight(self.w)
+        o.transpose_blockq(wq, sw)
+        t_quant = time.perf_counter() - t0
+        rows, flops = 0, 0
+        t1 = time.perf_counter()
+        while rows < 1 or (time.perf_counter() - t1 < gemm_budget_s and rows < 64):
+            r = rows % self.a_rows.shape[0]
+            o.gemm_mgrouped_full(self.a_rows[r:r + 1], np.ascontiguousarray(self.sa_rows[:, r:r + 1]),
+                                 wq, sw, np.array([0, 1], np.int32))
+            rows += 1
+            flops += 2 * self.wrows * K
+        t_gemm = time.perf_counter() - t1
+        desc = (f"fp64 GEMM of {rows} output rows x {self.wrows} cols x K={K} (expert {self.e}), "
+                f"permute+1x128 quantize of {self.ntok} tokens (top-{self.cfg.k}), 128x128 quantize "
+                f"and transpose of a [{self.wrows}x{K}] weight slab; 1 thread")
+        return flops / t_gemm / 1e12, self.q_bytes / t_quant / 1e9, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = W.CONFIGS[args.config]
+    sample = OracleSample(cfg)
+    times, tf_list, gb_list = [], [], []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        tf, gb, desc = sample.run(gemm_budget_s=2.0)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+            tf_list.append(tf)
+            gb_list.append(gb)
+    value = statistics.median(tf_list)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "description": cfg.description},
+        "quantize_gbs": statistics.median(gb_list),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
+    ap.add_argument("--config", default="dsv3", choices=sorted(W.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.config == "dsv3_bwd":
+        args.config = "dsv3"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    from fp8_fine_grained_permute_b200 import build as fbuild
+    from fp8_fine_grained_permute_b200 import fg8
+    if rank == 0:
+        fbuild.build()
+    if pg:
+        pg.barrier()
+    fg8.lib()
+
+    cfg = W.CONFIGS[args.config]
+    st = Step(cfg, dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            st.run(stream)
+    torch.cuda.synchronize()
+    if st.status.item() != 0:
+        raise RuntimeError(f"device status {fg8.status_name(st.status.item())}")
+
+    # ---------------- kernel-level timed region
+    marks = {}
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        st.run(stream, marks)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = clk.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    kern_ms = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in marks.items()}
+
+    pk = peaks()
+    fp8_peak = pk["bf16_sus"] * FP8_OVER_BF16
+    kernels = []
+    gemm_flops = gemm_ms = q_bytes = q_ms = 0.0
+    for name, (bound, amount) in st.work.items():
+        ms = kern_ms[name]
+        if bound == "tensor":
+            ach = amount / (ms * 1e-3) / 1e12
+            entry = {"kernel": name, "bound": "tensor", "ms": ms, "achieved": ach,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": ach / fp8_peak}
+            gemm_flops += amount
+            gemm_ms += ms
+            if name == "gemm_wgrad":      # fp32 output of E*N*K words is part of its floor
+                out_bytes = cfg.E * cfg.n_up * cfg.hidden * 4
+                entry["hbm_floor_ms"] = out_bytes / (pk["hbm_gbs"] * 1e9) * 1e3
+        else:
+            ach = amount / (ms * 1e-3) / 1e9
+            entry = {"kernel": name, "bound": "hbm", "ms": ms, "achieved": ach,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"]}
+            q_bytes += amount
+            q_ms += ms
+        entry["share"] = ms / ms_step
+        kernels.append(entry)
+    dom = max(kernels, key=lambda d: d["ms"])
+    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    quant_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    if pg:
+        t = torch.tensor([gemm_tflops, quant_gbs], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.SUM)
+        gemm_tflops, quant_gbs = float(t[0]), float(t[1])
+
+    # ---------------- end-to-end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        ins, outs = st.host_io()
+        h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+        d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                for h, d in ins:
+                    d.copy_(h, non_blocking=True)
+                st.run(stream)
+                for h, d in outs:
+                    h.copy_(d, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * gemm_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "GEMM FLOPs per step over the whole step time including pinned-host "
+                       "copies of X, ids, H, dY in and the forward output and dX out"}
+    if st.status.item() != 0:
+        raise RuntimeError(f"device status {fg8.status_name(st.status.item())}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, gb, desc = OracleSample(cfg).run(gemm_budget_s=10.0)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc,
+               "quantize_gbs": gb}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": gemm_tflops, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 x e4m3 -> f32 (GEMM); bf16 -> e4m3 (quantize)",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "description": cfg.description,
+                       "E": cfg.E, "T": cfg.T, "k": cfg.k, "hidden": cfg.hidden,
+                       "n_up": cfg.n_up, "inter": cfg.inter, "routed_rows": cfg.R,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (step working set > 50 GB)"},
+            "quantize_gbs": quant_gbs,
+            "gemm_frac_of_fp8_peak": gemm_tflops / world / fp8_peak,
+            "quantize_frac_of_hbm": quant_gbs / world / pk["hbm_gbs"],
+            "roofline": {"kernel": dom["kernel"], "bound": dom["bound"], "achieved": dom["achieved"],
+                         "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
+                         "traffic": None,
+                         "peak_source": f"{pk['source']}: HBM {pk['hbm_gbs']} GB/s; FP8 = "
+                                        f"{FP8_OVER_BF16} x sustained BF16 {pk['bf16_sus']} TFLOP/s"},
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clocks,
+            "gpu_launches": st.launches_per_step * args.steps,
+        }
+        print(json.dumps(line))
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

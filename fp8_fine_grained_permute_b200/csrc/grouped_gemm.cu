@@ -1,0 +1,557 @@
+// grouped_gemm.cu -- grouped FP8 GEMM with fine-grained scales on tcgen05.
+//
+// Computes, for every expert e (DeepSeek-V3 summary sec. 2.2: most GEMMs in
+// FP8 with 1x128 / 128x128 scaling and high-precision accumulation; Kanana-2
+// deep dive, devday.kr, FP8 paragraph):
+//     out[r][n] = sum_kb  sA(r,kb) * sB(n,kb) * sum_{k in block kb} A[r][k] * B[n][k]
+// The scales are arbitrary fp32 values, so they cannot be folded into the
+// tensor-core instruction (its block-scaled form takes power-of-two scales at
+// 32-element granularity).  Instead each 128-wide K block is multiplied on the
+// tensor core into its own TMEM partial (fp32), and the promotion warps add
+// partial * sA * sB into fp32 accumulators held in registers: the paged
+// design's "CUDA-core promotion", with the partial sums living in TMEM.
+//
+// CTA = one persistent worker per SM, 10 warps:
+//   warp 0      TMA producer: A tile 128x128 B and B tile 256x128 B per K block
+//               into a 4-stage ring (48 KB per stage), 128-byte swizzle.
+//   warp 1      TMEM allocator + MMA issuer: 4 x tcgen05.mma (M=128, N=256,
+//               K=32, E4M3 x E4M3 -> f32) per K block into one of two TMEM
+//               partial buffers (2 x 256 columns); tcgen05.commit frees the smem
+//               stage and publishes the partial.
+//   warps 2..9  promotion + epilogue: two warpgroups, one per 128-column half;
+//               thread = one output row; tcgen05.ld the partial, release the
+//               buffer, acc = fma(partial, sA*sB, acc); after the last K block
+//               convert and store the row segment.
+// Tiles are 128 rows x 256 columns; the tile list (expert, m-tile, n-tile) is
+// rebuilt on the device from the expert offsets, so offsets never travel to the
+// host.  Zero-row experts have no tiles (row-grouped mode); in the
+// contraction-grouped mode an expert with no tokens writes zeros.
+//
+// Every mbarrier wait is bounded (FG8_ERR_TIMEOUT in *status, then the roles
+// wind down and TMEM is released); the kernel never traps.
+#include <cuda.h>
+
+#include "fg8_common.cuh"
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = BM * BK;              // 16 KB
+constexpr uint32_t kBBytes = BN * BK;              // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;      // 320
+constexpr int kMaxE = 2048;
+constexpr uint32_t kTmemCols = 512;                // two partial buffers of BN columns
+
+// tcgen05 instruction descriptor (kind::f8f6f4): D = f32 (bits 4-5 = 1),
+// A = B = E4M3 (format 0), both K-major, N >> 3 in bits 17-22, M >> 4 in 24-28.
+constexpr uint32_t kIdesc =
+    (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr uint32_t kOffStages = 0;
+constexpr uint32_t kOffBars = kStages * kStageBytes;            // 196608
+constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;               // full, empty, tfull, tempty, drain
+constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;          // tmem slot, abort flag
+constexpr uint32_t kOffTiles = kOffMisc + 16;                   // int32 [kMaxE + 1]
+constexpr uint32_t kOffWarp = kOffTiles + 4 * (kMaxE + 4);      // int32 [36]
+constexpr uint32_t kSmemBytes = kOffWarp + 4 * 36 + 1024;       // + alignment slack
+
+struct GemmArgs {
+    const float* sa;
+    const float* sb;
+    const int32_t* offsets;
+    int64_t M_total;
+    int N, K, E;
+    int mode;       // FG8_GROUP_M / FG8_GROUP_K
+    int out_f32;
+    void* out;
+    int32_t* status;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+
+FG8_DEV uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+FG8_DEV void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+FG8_DEV void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+FG8_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+FG8_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase `parity` of `bar`.  Gives up when another role
+// has aborted or after kWaitLimitNs (then records FG8_ERR_TIMEOUT and raises
+// the CTA's abort flag).
+FG8_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                       int32_t* status) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = fg8::globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (fg8::globaltimer_ns() - t0 > fg8::kWaitLimitNs) {
+            fg8::set_status(status, FG8_ERR_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+FG8_DEV void tma_load_2d(const CUtensorMap* map, uint32_t dst, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// K-major operand tile in shared memory, 128-byte rows, 128-byte swizzle:
+// 8-row atoms 1024 bytes apart (stride byte offset), descriptor version 1.
+FG8_DEV uint64_t smem_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;                  // leading byte offset (unused with this swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset
+    d |= (uint64_t)1 << 46;                  // descriptor version
+    d |= (uint64_t)2 << 61;                  // SWIZZLE_128B
+    return d;
+}
+
+FG8_DEV void mma_e4m3(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n"
+        "}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+FG8_DEV void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive fp32 columns of TMEM -> 16 registers per thread
+FG8_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+FG8_DEV uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// tile schedule
+// ---------------------------------------------------------------------------
+
+struct Tile {
+    int e;
+    int rows_valid;     // rows of the tile that belong to the expert
+    int n0;             // first output column
+    int kx0;            // first contraction column of the operands
+    int nkb;            // 128-wide contraction blocks
+    int64_t rowA;       // first operand-A row
+    int64_t rowB;       // first operand-B row
+    int64_t out_row0;   // first output row
+};
+
+FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const GemmArgs& a, int nt) {
+    int lo = 0, hi = a.E;   // largest e with s_tiles[e] <= tile
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tiles[mid] <= tile) lo = mid; else hi = mid;
+    }
+    Tile T;
+    T.e = lo;
+    const int local = tile - s_tiles[lo];
+    const int mt = local / nt, ntile = local - mt * nt;
+    T.n0 = ntile * BN;
+    const int32_t o0 = a.offsets[lo], o1 = a.offsets[lo + 1];
+    if (a.mode == FG8_GROUP_M) {
+        T.rowA = (int64_t)o0 + (int64_t)mt * BM;
+        // rows past M_total (offsets inconsistent with the buffers) are never touched
+        T.rows_valid = (int)max((int64_t)0, min((int64_t)min(BM, (o1 - o0) - mt * BM),
+                                                a.M_total - T.rowA));
+        T.kx0 = 0;
+        T.nkb = a.K / BK;
+        T.rowB = (int64_t)lo * a.N + T.n0;
+        T.out_row0 = T.rowA;
+    } else {
+        T.rowA = (int64_t)mt * BM;
+        T.rows_valid = BM;
+        // contraction range clamped to the operands' width
+        T.kx0 = min(max(o0, 0), a.K) & ~(BK - 1);
+        T.nkb = max(0, min(o1, a.K) - T.kx0) / BK;
+        T.rowB = T.n0;
+        T.out_row0 = (int64_t)lo * a.M_total + T.rowA;
+    }
+    return T;
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+
+template <bool kGroupK>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + kOffBars;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    int32_t* s_tiles = reinterpret_cast<int32_t*>(smem + kOffTiles);
+    int32_t* s_warp = reinterpret_cast<int32_t*>(smem + kOffWarp);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nt = (a.N + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // tiles per expert -> exclusive prefix (in place)
+    for (int e = threadIdx.x; e < a.E; e += kThreads) {
+        const int32_t cnt = a.mode == FG8_GROUP_M
+                                ? (max(0, a.offsets[e + 1] - a.offsets[e]) + BM - 1) / BM
+                                : (int32_t)(a.M_total / BM);
+        s_tiles[e] = cnt * nt;
+    }
+    __syncthreads();
+    fg8::block_exclusive_scan(s_tiles, s_tiles, a.E, s_warp);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = s_tiles[a.E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const Tile T = decode_tile(tile, s_tiles, a, nt);
+                for (int kb = 0; kb < T.nkb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sA = sbase + kOffStages + stage * kStageBytes;
+                    mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
+                    tma_load_2d(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA);
+                    tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let copies already issued land before the CTA winds down
+                const uint32_t last = (stage + kStages - 1) % kStages;
+                const uint32_t lp = stage == 0 ? (phase ^ 1u) : phase;
+                const uint64_t t0 = fg8::globaltimer_ns();
+                while (!mbar_try_wait(full_bar(last), lp) &&
+                       fg8::globaltimer_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const Tile T = decode_tile(tile, s_tiles, a, nt);
+                for (int kb = 0; kb < T.nkb; ++kb) {
+                    if (!mbar_wait(tempty_bar(buf), bphase ^ 1u, abort_flag, a.status) ||
+                        !mbar_wait(full_bar(stage), phase, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sA = sbase + kOffStages + stage * kStageBytes;
+                    const uint32_t d = tmem_base + buf * BN;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        mma_e4m3(d, smem_desc(sA + 32 * kk), smem_desc(sA + kABytes + 32 * kk),
+                                 kk > 0 ? 1u : 0u);
+                    mma_commit(empty_bar(stage));
+                    mma_commit(tfull_bar(buf));
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    buf ^= 1u;
+                    if (buf == 0) bphase ^= 1u;
+                }
+            }
+            // all MMAs issued by this thread are complete once drain_bar flips
+            mma_commit(drain_bar);
+            const uint64_t t0 = fg8::globaltimer_ns();
+            while (!mbar_try_wait(drain_bar, 0) && fg8::globaltimer_ns() - t0 < 100000000ull) {
+            }
+        }
+    } else {
+        // ---------------------------------------------------- promotion + epilogue
+        const int ep = warp - 2;
+        const int half = ep >> 2;            // 128-column half of the tile
+        const int quarter = warp & 3;        // TMEM lane quarter this warp may access
+        const int r = 32 * quarter + lane;   // tile row owned by this thread
+        const int NB = a.N / 128, KBt = a.K / BK;
+        uint32_t buf = 0, bphase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const Tile T = decode_tile(tile, s_tiles, a, nt);
+            const bool row_ok = r < T.rows_valid;
+            const int col0 = T.n0 + 128 * half;
+            const bool col_ok = col0 < a.N;
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            const int kb0 = T.kx0 / BK;
+            for (int kb = 0; kb < T.nkb; ++kb) {
+                const float sav =
+                    row_ok ? __ldg(a.sa + (int64_t)(kb0 + kb) * a.M_total + T.rowA + r) : 0.0f;
+                float sbv = 0.0f;
+                if (!kGroupK && col_ok)
+                    sbv = __ldg(a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt + kb);
+                const float s = sav * sbv;
+                if (!mbar_wait(tfull_bar(buf), bphase, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * BN + 128 * half;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float p[16];
+                    tmem_ld16(taddr + 16 * ch, p);
+                    if (!kGroupK) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[16 * ch + i] = fmaf(p[i], s, acc[16 * ch + i]);
+                    } else {
+                        const float4* sbp = reinterpret_cast<const float4*>(
+                            a.sb + (int64_t)(kb0 + kb) * a.N + col0 + 16 * ch);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 c4 = col_ok ? __ldg(sbp + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            acc[16 * ch + 4 * i + 0] = fmaf(p[4 * i + 0] * c4.x, sav, acc[16 * ch + 4 * i + 0]);
+                            acc[16 * ch + 4 * i + 1] = fmaf(p[4 * i + 1] * c4.y, sav, acc[16 * ch + 4 * i + 1]);
+                            acc[16 * ch + 4 * i + 2] = fmaf(p[4 * i + 2] * c4.z, sav, acc[16 * ch + 4 * i + 2]);
+                            acc[16 * ch + 4 * i + 3] = fmaf(p[4 * i + 3] * c4.w, sav, acc[16 * ch + 4 * i + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(buf));
+                buf ^= 1u;
+                if (buf == 0) bphase ^= 1u;
+            }
+            if (!ok) break;
+            if (row_ok && col_ok) {
+                const int64_t orow = T.out_row0 + r;
+                if (a.out_f32) {
+                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                                          orow * a.N + col0);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                } else {
+                    uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) +
+                                                        orow * a.N + col0);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        o[i] = make_uint4(pack_bf16x2(acc[8 * i + 0], acc[8 * i + 1]),
+                                          pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                                          pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]),
+                                          pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D u8 matrix [rows][cols] (row stride = cols bytes), box rows x 128 bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const uint8_t* b,
+                                       const float* sb, const int32_t* offsets, int64_t M_total,
+                                       int N, int K, int E, int group_mode, int bscale_mode,
+                                       int out_dtype, void* out, int32_t* dev_status,
+                                       fg8_stream_t stream) {
+    if (!a || !sa || !b || !sb || !offsets || !out) return FG8_ERR_INVALID_ARG;
+    if (E < 1 || N < 128 || K < 128 || N % 128 || K % 128 || M_total < 0)
+        return FG8_ERR_INVALID_ARG;
+    if (E > kMaxE) return FG8_ERR_UNSUPPORTED;
+    if (out_dtype != FG8_OUT_BF16 && out_dtype != FG8_OUT_F32) return FG8_ERR_INVALID_ARG;
+    if (!fg8h::aligned16(a) || !fg8h::aligned16(b) || !fg8h::aligned16(out) ||
+        !fg8h::aligned16(sb) || (reinterpret_cast<uintptr_t>(sa) & 3) ||
+        (reinterpret_cast<uintptr_t>(offsets) & 3))
+        return FG8_ERR_INVALID_ARG;
+    if (M_total > INT32_MAX) return FG8_ERR_UNSUPPORTED;
+
+    const int64_t nt = (N + BN - 1) / BN;
+    int64_t max_tiles;
+    CUtensorMap mA, mB;
+    if (group_mode == FG8_GROUP_M) {
+        if (bscale_mode != FG8_BSCALE_BLOCK128) return FG8_ERR_UNSUPPORTED;
+        if (M_total == 0) return FG8_OK;
+        if ((int64_t)E * N > INT32_MAX) return FG8_ERR_UNSUPPORTED;
+        max_tiles = (M_total / BM + E) * nt;
+        if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||
+            !make_map(&mB, b, (uint64_t)E * N, (uint64_t)K, BN))
+            return FG8_ERR_CUDA;
+    } else if (group_mode == FG8_GROUP_K) {
+        if (bscale_mode != FG8_BSCALE_ROW128) return FG8_ERR_UNSUPPORTED;
+        if (M_total % 128) return FG8_ERR_INVALID_ARG;
+        if (M_total == 0) return FG8_OK;
+        max_tiles = (int64_t)E * (M_total / BM) * nt;
+        if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||
+            !make_map(&mB, b, (uint64_t)N, (uint64_t)K, BN))
+            return FG8_ERR_CUDA;
+    } else {
+        return FG8_ERR_INVALID_ARG;
+    }
+    if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
+
+    auto kern = group_mode == FG8_GROUP_K ? grouped_gemm_kernel<true> : grouped_gemm_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess)
+        return FG8_ERR_CUDA;
+    GemmArgs args;
+    args.sa = sa;
+    args.sb = sb;
+    args.offsets = offsets;
+    args.M_total = M_total;
+    args.N = N;
+    args.K = K;
+    args.E = E;
+    args.mode = group_mode;
+    args.out_f32 = out_dtype == FG8_OUT_F32;
+    args.out = out;
+    args.status = dev_status;
+    int64_t grid = fg8h::num_sms();
+    if (grid > max_tiles) grid = max_tiles;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, kThreads, kSmemBytes, (cudaStream_t)stream>>>(mA, mB, args);
+    return fg8h::launch_status();
+}

@@ -310,3 +310,61 @@ def gen_dy(cfg: MoEConfig, device="cpu", row0: int = 0, rows: int | None = None)
     rows = cfg.R - row0 if rows is None else rows
     return gen_grad_bf16((rows, cfg.n_up), cfg.seed, SID_DY, device,
                          index_offset=row0 * cfg.n_up)
+
+
+# --------------------------------------------------------------------------
+# direct FP8 operands (for GEMM / transpose parity independent of quantization)
+# --------------------------------------------------------------------------
+
+def finite_e4m3_codes() -> torch.Tensor:
+    """The 254 finite E4M3 bit patterns (all but S.1111.111), as uint8."""
+    c = torch.arange(256, dtype=torch.int32)
+    keep = (c & 0x7F) != 0x7F
+    return c[keep].to(torch.uint8)
+
+
+@functools.lru_cache(maxsize=None)
+def _scale_table(lo_exp: int, hi_exp: int) -> torch.Tensor:
+    """2^16 fp32 values log-uniform in [2^lo_exp, 2^hi_exp)."""
+    n = 1 << 16
+    e = lo_exp + (hi_exp - lo_exp) * (torch.arange(n, dtype=torch.float64) + 0.5) / n
+    return torch.exp2(e).to(torch.float32)
+
+
+def gen_e4m3_codes(shape, seed: int, sid: int, device="cpu", index_offset: int = 0,
+                   chunk: int = 1 << 26) -> torch.Tensor:
+    """uint8 tensor of uniformly drawn finite E4M3 codes."""
+    numel = math.prod(shape)
+    codes = finite_e4m3_codes().to(device)
+    out = torch.empty(numel, dtype=torch.uint8, device=device)
+    for s in range(0, numel, chunk):
+        n = min(chunk, numel - s)
+        idx = torch.arange(index_offset + s, index_offset + s + n, dtype=torch.int64, device=device)
+        out[s:s + n] = codes[hash_index(idx, seed, sid) % codes.numel()]
+    return out.view(*shape)
+
+
+def gen_bytes(shape, seed: int, sid: int, device="cpu", index_offset: int = 0,
+              chunk: int = 1 << 26) -> torch.Tensor:
+    """uint8 tensor of uniform random bytes."""
+    numel = math.prod(shape)
+    out = torch.empty(numel, dtype=torch.uint8, device=device)
+    for s in range(0, numel, chunk):
+        n = min(chunk, numel - s)
+        idx = torch.arange(index_offset + s, index_offset + s + n, dtype=torch.int64, device=device)
+        out[s:s + n] = (hash_index(idx, seed, sid) & 0xFF).to(torch.uint8)
+    return out.view(*shape)
+
+
+def gen_bytes_at(idx: torch.Tensor, seed: int, sid: int) -> torch.Tensor:
+    """The bytes gen_bytes draws at arbitrary flat indices."""
+    return (hash_index(idx, seed, sid) & 0xFF).to(torch.uint8)
+
+
+def gen_scales(shape, seed: int, sid: int, device="cpu", lo_exp: int = -12, hi_exp: int = 0,
+               index_offset: int = 0) -> torch.Tensor:
+    """fp32 tensor of positive scales, log-uniform in [2^lo_exp, 2^hi_exp)."""
+    numel = math.prod(shape)
+    tab = _scale_table(lo_exp, hi_exp).to(device)
+    idx = torch.arange(index_offset, index_offset + numel, dtype=torch.int64, device=device)
+    return tab[hash_index(idx, seed, sid) >> 16].view(*shape)

@@ -1,0 +1,191 @@
+/*
+ * fg8.h -- C ABI of libfg8: FP8 fine-grained quantization for MoE expert
+ * layers on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow two pages:
+ *  [K2] "Kakao Kanana-2 pre-training deep dive" (devday.kr), the FP8 paragraph:
+ *       fine-grained FP8 scaling with 1x128 activation tiles and 128x128
+ *       weight blocks; one MoE quantization kernel for all experts instead of
+ *       one expert after another; a kernel that transposes block-quantized
+ *       weights for backward, so only the forward FP8 weight is stored.
+ *  [DS] "DeepSeek-V3 summary" (theinnovators.zone), sec. 2.1 (sigmoid
+ *       affinity, top-K routing, per-expert bias, no token dropping) and
+ *       sec. 2.2 "FP8 mixed precision training" (most GEMMs in FP8, 1x128 /
+ *       128x128 tile/block quantization, high-precision accumulation).
+ *
+ * Numerics (one reading of the pages, which fix neither format nor formula):
+ * FP8 is OCP E4M3FN.  For each tile or block with largest magnitude amax,
+ *     s = fp32(amax / 448)   (s = 1 when amax == 0),
+ *     q = E4M3(fp32(x / s))  round to nearest, ties to even, saturating at
+ *                            +-448, sign of zero kept.
+ * s is the dequantization multiplier: x ~= q * s.  NaN/Inf inputs are outside
+ * the contract (their outputs are unspecified).
+ *
+ * Conventions for every call:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, never synchronizes the stream and keeps no state
+ *    between calls, so calls on different streams with disjoint buffers are
+ *    independent.  `stream` is a cudaStream_t (NULL = the legacy stream).
+ *  - bf16 data is passed as uint16_t bit patterns.  FP8 data as uint8_t.
+ *  - Calls are asynchronous.  Argument errors are found on the host and
+ *    returned immediately (nothing is launched).  Launch failures return
+ *    FG8_ERR_CUDA.  Conditions only the device can see (an expert id out of
+ *    range, a bounded wait that ran out) are written to *dev_status (a device
+ *    int32 that the caller zeroes once and reads after synchronizing); the
+ *    library sets it to the first such fg8_status and never clears it.
+ *    Kernels never trap.
+ *  - Buffers that TMA reads (the GEMM operands) and every FP8/bf16 buffer
+ *    must be 16-byte aligned; row strides are implied by the sizes.
+ */
+#ifndef FG8_H
+#define FG8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FG8_OK = 0,
+    FG8_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment   */
+    FG8_ERR_UNSUPPORTED = 2,   /* valid but not implemented combination  */
+    FG8_ERR_CUDA = 3,          /* a CUDA runtime/launch error            */
+    FG8_ERR_BAD_EXPERT_ID = 4, /* device: an id outside [0, E) was met   */
+    FG8_ERR_TIMEOUT = 5        /* device: a bounded wait ran out         */
+} fg8_status;
+
+typedef enum { FG8_ROWWISE = 1, FG8_COLWISE = 2 } fg8_act_layout;
+typedef enum { FG8_OUT_BF16 = 0, FG8_OUT_F32 = 1 } fg8_out_dtype;
+typedef enum { FG8_GROUP_M = 0, FG8_GROUP_K = 1 } fg8_group_mode;
+typedef enum { FG8_BSCALE_BLOCK128 = 0, FG8_BSCALE_ROW128 = 1 } fg8_bscale_mode;
+
+typedef void* fg8_stream_t; /* cudaStream_t */
+
+/*
+ * fg8_quantize_act -- 1x128 activation quantization to E4M3 with one fp32
+ * scale per tile, fused with the token-to-expert permute, all experts in one
+ * launch ([K2] FP8 paragraph; [DS] sec. 2.1 no token dropping, sec. 2.2
+ * 1x128 tiles).
+ *
+ * layout = FG8_ROWWISE, topk_ids != NULL  (forward dispatch):
+ *   x          bf16  [T][K], K % 128 == 0
+ *   topk_ids   int32 [T][k], expert ids in [0, E)
+ *   xq         E4M3  [R][K], R = T*k; rows grouped by expert, experts in
+ *              ascending order, inside an expert by ascending (token, slot)
+ *   sa         fp32  [K/128][R]: sa[kb*R + r] is the scale of row r, K block kb
+ *   row_token  int32 [R]:   token of each row
+ *   token_row  int32 [T*k]: row of each (token, slot); -1 for a bad id
+ *   offsets_out int32 [E+1]: expert e owns rows [offsets_out[e], offsets_out[e+1])
+ *   workspace  >= fg8_quantize_act_workspace(T, k, E) bytes, 16-byte aligned
+ *   Each token row is read once and its codes written to its k rows.  An id
+ *   outside [0, E) sets *dev_status = FG8_ERR_BAD_EXPERT_ID; that pair gets
+ *   no row (the tail rows of xq/sa/row_token stay unwritten).
+ *   This mode uses a cooperative launch (all CTAs resident) with grid-wide
+ *   barriers whose waits are bounded (FG8_ERR_TIMEOUT in *dev_status).
+ *   Calls that share one workspace must not overlap on the GPU.
+ *
+ * layout = FG8_ROWWISE, topk_ids == NULL  (rows already in expert order):
+ *   x [T][K] -> xq [T][K], sa [K/128][T]; k must be 1; E, offsets and index
+ *   maps are ignored (may be 0/NULL); workspace may be NULL.
+ *
+ * layout = FG8_COLWISE  (weight-gradient operands: 1x128 along the token axis)
+ *   Logical rows r in [0, R), R = T*k, are grouped by expert through
+ *   offsets_in [E+1] (device, offsets_in[E] == R).  If row_token != NULL it
+ *   is an INPUT [R] and logical row r is x[row_token[r]] (x has T rows);
+ *   otherwise k must be 1 and logical row r is x[r].  Each expert's rows are
+ *   cut into tiles of 128 consecutive rows, the last one zero-padded; every
+ *   (column, tile) gets one scale (padding takes no part in amax, and is
+ *   written as code 0x00).  With P = fg8_colwise_capacity(R, E):
+ *   xqT        E4M3 [K][P]: token axis contiguous; expert e occupies columns
+ *              [offsets_out[e], offsets_out[e+1]) of each row
+ *   saT        fp32 [P/128][K]: saT[(p/128)*K + c]
+ *   offsets_out int32 [E+1]: padded offsets, sum of ceil(T_e/128)*128
+ *   Columns past offsets_out[E] are not written.  xq, sa, token_row and
+ *   workspace are unused.
+ */
+fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
+                            const int32_t* topk_ids, int k, int E,
+                            const int32_t* offsets_in, int layout,
+                            uint8_t* xq, float* sa,
+                            int32_t* row_token, int32_t* token_row, int32_t* offsets_out,
+                            uint8_t* xqT, float* saT,
+                            void* workspace, size_t ws_bytes,
+                            int32_t* dev_status, fg8_stream_t stream);
+
+/* Workspace bytes needed by fg8_quantize_act in the permuting mode. */
+size_t fg8_quantize_act_workspace(int64_t T, int k, int E);
+
+/* Width P of the column-wise buffers for R logical rows over E experts:
+ * round_up(R + 127*E, 128). */
+int64_t fg8_colwise_capacity(int64_t R, int E);
+
+/*
+ * fg8_quantize_weight -- 128x128 block quantization of the weights of all
+ * experts in one launch ([K2] FP8 paragraph; [DS] sec. 2.2 128x128 blocks).
+ *   w   bf16 [E][N][K], N % 128 == 0, K % 128 == 0
+ *   wq  E4M3 [E][N][K]
+ *   sw  fp32 [E][N/128][K/128]
+ */
+fg8_status fg8_quantize_weight(const uint16_t* w, int E, int N, int K,
+                               uint8_t* wq, float* sw, fg8_stream_t stream);
+
+/*
+ * fg8_transpose_blockq -- transpose an already block-quantized weight and its
+ * scale grid for backward, so only the forward FP8 copy is stored ([K2] FP8
+ * paragraph, last sentence).  Pure byte/scale moves: because the blocks are
+ * square, dequant(transpose(Q)) == transpose(dequant(Q)) exactly.
+ *   wq  E4M3 [E][N][K] -> wqT E4M3 [E][K][N]
+ *   sw  fp32 [E][N/128][K/128] -> swT fp32 [E][K/128][N/128]
+ */
+fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N, int K,
+                                uint8_t* wqT, float* swT, fg8_stream_t stream);
+
+/*
+ * fg8_grouped_gemm -- grouped FP8 GEMM with fine-grained scales: at every
+ * 128-wide K step the tensor-core partial product is promoted into an fp32
+ * accumulator with the activation tile scale and the weight block scale
+ * ([DS] sec. 2.2 most GEMMs in FP8, high-precision accumulation; [K2] FP8
+ * paragraph).  Runs on tcgen05 tensor cores (TMEM accumulators, TMA loads).
+ * out[r][n] = sum_kb sA(r,kb) * sB(n,kb) * sum_{k in kb} A[r][k] * B[n][k].
+ *
+ * group_mode = FG8_GROUP_M (forward / dgrad; variable rows per expert):
+ *   a        E4M3 [M_total][K]; sa fp32 [K/128][M_total]
+ *   b        E4M3 [E][N][K] (K-major, e.g. fg8_quantize_weight's wq, or
+ *            fg8_transpose_blockq's wqT for dgrad)
+ *   sb       fp32 [E][N/128][K/128] (bscale_mode = FG8_BSCALE_BLOCK128)
+ *   offsets  int32 [E+1] on the device: expert e owns rows
+ *            [offsets[e], offsets[e+1]); offsets[E] <= M_total
+ *   out      [M_total][N] bf16 or fp32; rows outside [0, offsets[E]) are
+ *            not written.  An expert with no rows costs nothing.
+ *   N % 128 == 0, K % 128 == 0.
+ *
+ * group_mode = FG8_GROUP_K (weight gradient; variable contraction per expert):
+ *   a        E4M3 [M_total][K], sa fp32 [K/128][M_total]
+ *   b        E4M3 [N][K],       sb fp32 [K/128][N] (bscale_mode = FG8_BSCALE_ROW128)
+ *   offsets  int32 [E+1] on the device, multiples of 128, offsets[E] <= K
+ *            (fg8_quantize_act COLWISE's offsets_out; K = its capacity P)
+ *   out      [E][M_total][N]: out[e] = sum over columns [offsets[e],
+ *            offsets[e+1]) of the contraction; an expert with no columns gets
+ *            zeros.  M_total % 128 == 0, N % 128 == 0, K % 128 == 0.
+ *
+ * The fp32 output is the accumulator; the bf16 output is its round-to-
+ * nearest-even conversion.  dev_status may be NULL only if no device-side
+ * condition needs reporting is acceptable to the caller (bounded waits still
+ * end the kernel).
+ */
+fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa,
+                            const uint8_t* b, const float* sb,
+                            const int32_t* offsets, int64_t M_total, int N, int K, int E,
+                            int group_mode, int bscale_mode, int out_dtype, void* out,
+                            int32_t* dev_status, fg8_stream_t stream);
+
+/* Static string naming a status. */
+const char* fg8_status_string(fg8_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FG8_H */
