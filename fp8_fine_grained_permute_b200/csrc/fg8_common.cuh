@@ -50,43 +50,35 @@ FG8_DEV float tile_scale(float amax) {
     return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
 }
 
-// Per-tile context for the fast path of fp32(x / s).
+// Per-tile context of the E4M3 quantization.
 //
-// The product y' = x * rcp(s) differs from the correctly rounded quotient
-// fp32(x / s) by a few fp32 ulps.  E4M3 rounding of a value in the normal
-// E4M3 range (|y| >= 2^-6) looks only at the top three fraction bits and
-// compares the low 20 fraction bits with the midpoint pattern 0x80000; a
-// few-ulp error changes the E4M3 result only if y' lies within those ulps of
-// a midpoint.  So: if y' is more than 128 ulps away from every midpoint and
-// |y'| >= 2^-6, E4M3(y') == E4M3(fp32(x / s)) exactly; otherwise (and for
-// subnormal scales, whose reciprocal overflows) the IEEE division is used.
-// The 128-ulp window covers any reciprocal with relative error below 2^-17;
-// the hardware approximation is within a few ulps.
+// The exact code of an element is E4M3(z) with z = fp32(x / s) (IEEE
+// division).  Fast path: with r ~ 1/s, E4M3 rounding is monotonic, so if the
+// two products x * r(1 - eps) and x * r(1 + eps) get the same code, and the
+// interval between them contains z, that shared code is E4M3(z).  r is the
+// hardware reciprocal refined by one Newton-Raphson step, r <- r + r (1 - s r),
+// so |r - 1/s| <= 2^-23 / s; with the two roundings of the products and the
+// rounding of z the interval holds z whenever eps > 5 * 2^-24, and eps = 2^-18
+// leaves a factor of ten.  Elements whose two codes differ (a rounding midpoint
+// lies inside the interval: about 1 in 8000) and tiles whose scale is
+// subnormal (its reciprocal would overflow) take the IEEE division.
 struct QScale {
-    float s;     // scale (dequantization multiplier)
-    float r;     // approximate 1/s
-    bool exact;  // take the division for every element
+    float s;        // scale (dequantization multiplier)
+    float r_lo;     // fp32(r * (1 - 2^-18))
+    float r_hi;     // fp32(r * (1 + 2^-18))
+    bool exact;     // take the division for every element of the tile
 };
 
 FG8_DEV QScale make_qscale(float s) {
     QScale q;
     q.s = s;
-    float r;
-    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(s));
-    q.r = r;
-    q.exact = !(s >= 1.17549435e-38f) || !(fabsf(r) <= 3.0e38f);
+    float r0;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r0) : "f"(s));
+    const float r = fmaf(r0, fmaf(-s, r0, 1.0f), r0);   // Newton-Raphson step
+    q.r_lo = __fmul_rn(r, 1.0f - 0x1p-18f);
+    q.r_hi = __fmul_rn(r, 1.0f + 0x1p-18f);
+    q.exact = !(s >= 1.17549435e-38f);                   // subnormal scale
     return q;
-}
-
-// fp32 value whose E4M3 rounding equals that of fp32(x / s).
-FG8_DEV float quot(float x, const QScale& q) {
-    float y = __fmul_rn(x, q.r);
-    uint32_t b = __float_as_uint(y) & 0x7FFFFFFFu;
-    uint32_t low = b & 0xFFFFFu;
-    bool near_mid = (low - (0x80000u - 128u)) <= 256u;
-    bool small = (b < 0x3C800000u) && (b != 0u);      // 0 < |y| < 2^-6
-    if (q.exact || near_mid || small) y = __fdiv_rn(x, q.s);
-    return y;
 }
 
 // Two fp32 -> two E4M3 (RNE, saturating to +-448): `lo` in bits 7..0.
@@ -96,23 +88,67 @@ FG8_DEV uint32_t cvt_e4m3x2(float lo, float hi) {
     return (uint32_t)r;
 }
 
+FG8_DEV uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+FG8_DEV uint32_t cvt_e4m3x2(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return cvt_e4m3x2(lo, hi);
+}
+
+FG8_DEV uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// E4M3 codes of (x0, x1) with scale context q, x0 in bits 7..0.
+FG8_DEV uint32_t quant_pair(float x0, float x1, const QScale& q) {
+    if (!q.exact) {
+        const uint64_t x = pack_f32x2(x0, x1);
+        const uint32_t lo = cvt_e4m3x2(mul_f32x2(x, pack_f32x2(q.r_lo, q.r_lo)));
+        const uint32_t hi = cvt_e4m3x2(mul_f32x2(x, pack_f32x2(q.r_hi, q.r_hi)));
+        if (lo == hi) return lo;
+    }
+    return cvt_e4m3x2(__fdiv_rn(x0, q.s), __fdiv_rn(x1, q.s));
+}
+
 // Quantize 8 bf16 values (one uint4) with scale context q -> 8 codes (uint2).
+// The fast-path check is made once for all 8 codes, so the rare exact path
+// costs one (usually not taken) branch per 8 elements.
 FG8_DEV uint2 quant8(const uint4& v, const QScale& q) {
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if (!q.exact) {
+        const uint64_t rl = pack_f32x2(q.r_lo, q.r_lo), rh = pack_f32x2(q.r_hi, q.r_hi);
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint64_t x = pack_f32x2(bf16_lo(w[i]), bf16_hi(w[i]));
+            lo[i] = cvt_e4m3x2(mul_f32x2(x, rl));
+            hi[i] = cvt_e4m3x2(mul_f32x2(x, rh));
+        }
+        const uint2 cl = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+        const uint2 ch = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+        if (cl.x == ch.x && cl.y == ch.y) return cl;
+    }
     uint32_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        c[i] = cvt_e4m3x2(quot(bf16_lo(w[i]), q), quot(bf16_hi(w[i]), q));
+        c[i] = cvt_e4m3x2(__fdiv_rn(bf16_lo(w[i]), q.s), __fdiv_rn(bf16_hi(w[i]), q.s));
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// max |x| over 8 bf16 values
+// max |x| over 8 bf16 values: magnitudes of non-NaN floats order like their
+// bit patterns, so a 16-bit SIMD unsigned max over the sign-cleared words is exact.
 FG8_DEV float amax8(const uint4& v) {
-    float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
-    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
-    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))));
-    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))));
-    return m;
+    uint32_t m = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    const uint32_t h = max(m & 0xFFFFu, m >> 16);
+    return __uint_as_float(h << 16);
 }
 
 // ---------------------------------------------------------------------------

@@ -40,9 +40,10 @@ constexpr int kStages = 4;
 constexpr uint32_t kABytes = BM * BK;              // 16 KB
 constexpr uint32_t kBBytes = BN * BK;              // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;      // 320
-constexpr int kMaxE = 2048;
+constexpr int kEpiWarps = 8;                       // two promotion warpgroups
+constexpr int kCtrlWarps = 4;                      // warpgroup 0: TMA, MMA, 2 idle warps
+constexpr int kThreads = 32 * (kCtrlWarps + kEpiWarps);   // 384
+constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;                // two partial buffers of BN columns
 
 // tcgen05 instruction descriptor (kind::f8f6f4): D = f32 (bits 4-5 = 1),
@@ -57,7 +58,21 @@ constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;               // full, empty, 
 constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;          // tmem slot, abort flag
 constexpr uint32_t kOffTiles = kOffMisc + 16;                   // int32 [kMaxE + 1]
 constexpr uint32_t kOffWarp = kOffTiles + 4 * (kMaxE + 4);      // int32 [36]
-constexpr uint32_t kSmemBytes = kOffWarp + 4 * 36 + 1024;       // + alignment slack
+// epilogue staging: per promotion warp 32 rows x 16 words (+4 words padding)
+constexpr int kStageWords = 20;
+constexpr uint32_t kStagePerWarp = 32 * kStageWords * 4;         // 2560 bytes
+constexpr uint32_t kOffStage = (kOffWarp + 4 * 36 + 15) & ~15u;
+// contraction-grouped mode: per K block the producer also copies the 128 row
+// scales of A and the 256 column scales of B into a ring of kScaleSlots slots.
+// A slot is rewritten kScaleSlots K blocks later, i.e. only after the MMA of
+// K block c+2 has taken the TMEM buffer that the promotion of K block c (the
+// slot's reader) released, so kStages + 2 slots never race.
+constexpr int kScaleSlots = kStages + 2;
+constexpr uint32_t kScaleSlotBytes = 4 * (BM + BN);            // 1536
+constexpr uint32_t kOffScales = kOffStage + kEpiWarps * kStagePerWarp;
+constexpr uint32_t kSmemBytes = kOffScales + kScaleSlots * kScaleSlotBytes + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert((kStageWords * 4) % 16 == 0 && kOffStage % 16 == 0, "staged rows are 16-byte vectors");
 
 struct GemmArgs {
     const float* sa;
@@ -134,6 +149,14 @@ FG8_DEV void tma_load_2d(const CUtensorMap* map, uint32_t dst, uint32_t bar, int
         : "memory");
 }
 
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0)
+FG8_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 // K-major operand tile in shared memory, 128-byte rows, 128-byte swizzle:
 // 8-row atoms 1024 bytes apart (stride byte offset), descriptor version 1.
 FG8_DEV uint64_t smem_desc(uint32_t addr) {
@@ -165,6 +188,22 @@ FG8_DEV void mma_commit(uint32_t bar) {
 
 FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns of TMEM -> 32 registers per thread
+FG8_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 
 // 32 lanes x 16 consecutive fp32 columns of TMEM -> 16 registers per thread
 FG8_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
@@ -300,7 +339,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
-            uint32_t stage = 0, phase = 0;
+            uint32_t stage = 0, phase = 0, sc = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 const Tile T = decode_tile(tile, s_tiles, a, nt);
@@ -310,7 +349,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         break;
                     }
                     const uint32_t sA = sbase + kOffStages + stage * kStageBytes;
-                    mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
+                    if (kGroupK) {
+                        const int kbg = T.kx0 / BK + kb;
+                        const uint32_t sb_bytes = 4u * (uint32_t)min(BN, a.N - T.n0);
+                        const uint32_t slot = sbase + kOffScales + (sc % kScaleSlots) * kScaleSlotBytes;
+                        mbar_arrive_expect_tx(full_bar(stage), kStageBytes + 4 * BM + sb_bytes);
+                        bulk_load(slot, a.sa + (int64_t)kbg * a.M_total + T.rowA, 4 * BM, full_bar(stage));
+                        bulk_load(slot + 4 * BM, a.sb + (int64_t)kbg * a.N + T.n0, sb_bytes, full_bar(stage));
+                        ++sc;
+                    } else {
+                        mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
+                    }
                     tma_load_2d(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA);
                     tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
                     if (++stage == kStages) {
@@ -365,31 +414,45 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             while (!mbar_try_wait(drain_bar, 0) && fg8::globaltimer_ns() - t0 < 100000000ull) {
             }
         }
-    } else {
+    } else if (warp >= kCtrlWarps) {
         // ---------------------------------------------------- promotion + epilogue
-        const int ep = warp - 2;
+        const int ep = warp - kCtrlWarps;
         const int half = ep >> 2;            // 128-column half of the tile
         const int quarter = warp & 3;        // TMEM lane quarter this warp may access
         const int r = 32 * quarter + lane;   // tile row owned by this thread
         const int NB = a.N / 128, KBt = a.K / BK;
-        uint32_t buf = 0, bphase = 0;
+        uint32_t buf = 0, bphase = 0, sc = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
             const Tile T = decode_tile(tile, s_tiles, a, nt);
             const bool row_ok = r < T.rows_valid;
             const int col0 = T.n0 + 128 * half;
             const bool col_ok = col0 < a.N;
-            float acc[128];
+            float2 acc[64];   // columns 2i, 2i + 1 of this thread's 128-column half
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
             const int kb0 = T.kx0 / BK;
+            // row-grouped mode: scales prefetched two K blocks ahead in registers
+            const float* sa_p = a.sa + T.rowA + r;
+            const float* sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
+            float sa_c = 0.f, sa_n = 0.f, sb_c = 0.f, sb_n = 0.f;
+            if (!kGroupK) {
+                if (row_ok && T.nkb > 0) sa_c = __ldg(sa_p);
+                if (row_ok && T.nkb > 1) sa_n = __ldg(sa_p + a.M_total);
+                if (col_ok && T.nkb > 0) sb_c = __ldg(sb_p);
+                if (col_ok && T.nkb > 1) sb_n = __ldg(sb_p + 1);
+            }
             for (int kb = 0; kb < T.nkb; ++kb) {
-                const float sav =
-                    row_ok ? __ldg(a.sa + (int64_t)(kb0 + kb) * a.M_total + T.rowA + r) : 0.0f;
-                float sbv = 0.0f;
-                if (!kGroupK && col_ok)
-                    sbv = __ldg(a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt + kb);
-                const float s = sav * sbv;
+                float s = 0.f;
+                if (!kGroupK) {
+                    s = sa_c * sb_c;
+                    sa_c = sa_n;
+                    sb_c = sb_n;
+                    if (kb + 2 < T.nkb) {
+                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 2) * a.M_total);
+                        if (col_ok) sb_n = __ldg(sb_p + kb + 2);
+                    }
+                }
                 if (!mbar_wait(tfull_bar(buf), bphase, abort_flag, a.status)) {
                     ok = false;
                     break;
@@ -397,23 +460,41 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 tc_fence_after();
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * BN + 128 * half;
+                if (!kGroupK) {
+                    const float2 s2 = make_float2(s, s);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float p[16];
-                    tmem_ld16(taddr + 16 * ch, p);
-                    if (!kGroupK) {
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t p[32];
+                        tmem_ld32(taddr + 32 * ch, p);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[16 * ch + i] = fmaf(p[i], s, acc[16 * ch + i]);
-                    } else {
-                        const float4* sbp = reinterpret_cast<const float4*>(
-                            a.sb + (int64_t)(kb0 + kb) * a.N + col0 + 16 * ch);
+                        for (int i = 0; i < 16; ++i)
+                            acc[16 * ch + i] = __ffma2_rn(
+                                make_float2(__uint_as_float(p[2 * i]), __uint_as_float(p[2 * i + 1])),
+                                s2, acc[16 * ch + i]);
+                    }
+                } else {
+                    // scales of this K block, staged by the producer
+                    const float* slot = reinterpret_cast<const float*>(
+                        smem + kOffScales + (sc % kScaleSlots) * kScaleSlotBytes);
+                    ++sc;
+                    const float sa_r = slot[r];
+                    const float2 sa2 = make_float2(sa_r, sa_r);
+                    const float4* sbv = reinterpret_cast<const float4*>(slot + BM + 128 * half);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 c4 = col_ok ? __ldg(sbp + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-                            acc[16 * ch + 4 * i + 0] = fmaf(p[4 * i + 0] * c4.x, sav, acc[16 * ch + 4 * i + 0]);
-                            acc[16 * ch + 4 * i + 1] = fmaf(p[4 * i + 1] * c4.y, sav, acc[16 * ch + 4 * i + 1]);
-                            acc[16 * ch + 4 * i + 2] = fmaf(p[4 * i + 2] * c4.z, sav, acc[16 * ch + 4 * i + 2]);
-                            acc[16 * ch + 4 * i + 3] = fmaf(p[4 * i + 3] * c4.w, sav, acc[16 * ch + 4 * i + 3]);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t p[32];
+                        tmem_ld32(taddr + 32 * ch, p);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 c4 = col_ok ? sbv[8 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                            const float2 w0 = __fmul2_rn(make_float2(c4.x, c4.y), sa2);
+                            const float2 w1 = __fmul2_rn(make_float2(c4.z, c4.w), sa2);
+                            acc[16 * ch + 2 * i] = __ffma2_rn(
+                                make_float2(__uint_as_float(p[4 * i]), __uint_as_float(p[4 * i + 1])), w0,
+                                acc[16 * ch + 2 * i]);
+                            acc[16 * ch + 2 * i + 1] = __ffma2_rn(
+                                make_float2(__uint_as_float(p[4 * i + 2]), __uint_as_float(p[4 * i + 3])), w1,
+                                acc[16 * ch + 2 * i + 1]);
                         }
                     }
                 }
@@ -424,23 +505,54 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (buf == 0) bphase ^= 1u;
             }
             if (!ok) break;
-            if (row_ok && col_ok) {
-                const int64_t orow = T.out_row0 + r;
+            // Epilogue: 16 words of each row at a time go through this warp's
+            // staging rows, then every store instruction writes 8 rows x 64
+            // contiguous bytes (whole sectors) instead of 32 scattered pieces.
+            if (col_ok) {
+                uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kOffStage) + ep * 32 * kStageWords;
+                uint4* my_row = reinterpret_cast<uint4*>(stg + lane * kStageWords);
+                const int sub = ((lane >> 2) & 1) * 4 + (lane >> 3);  // rows g*8+sub, conflict-free
+                const int quad = lane & 3;
                 if (a.out_f32) {
-                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
-                                                          orow * a.N + col0);
+                    float* ob = static_cast<float*>(a.out) + col0 + 4 * quad;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                    for (int ch = 0; ch < 8; ++ch) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            my_row[q] = make_uint4(__float_as_uint(acc[8 * ch + 2 * q].x),
+                                                   __float_as_uint(acc[8 * ch + 2 * q].y),
+                                                   __float_as_uint(acc[8 * ch + 2 * q + 1].x),
+                                                   __float_as_uint(acc[8 * ch + 2 * q + 1].y));
+                        __syncwarp();
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int rr = 8 * g + sub;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
+                            if (32 * quarter + rr < T.rows_valid)
+                                *reinterpret_cast<uint4*>(ob + (T.out_row0 + 32 * quarter + rr) * a.N + 16 * ch) = v;
+                        }
+                        __syncwarp();
+                    }
                 } else {
-                    uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) +
-                                                        orow * a.N + col0);
+                    uint16_t* ob = static_cast<uint16_t*>(a.out) + col0 + 8 * quad;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        o[i] = make_uint4(pack_bf16x2(acc[8 * i + 0], acc[8 * i + 1]),
-                                          pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
-                                          pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]),
-                                          pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+                    for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            my_row[q] = make_uint4(pack_bf16x2(acc[16 * ch + 4 * q + 0].x, acc[16 * ch + 4 * q + 0].y),
+                                                   pack_bf16x2(acc[16 * ch + 4 * q + 1].x, acc[16 * ch + 4 * q + 1].y),
+                                                   pack_bf16x2(acc[16 * ch + 4 * q + 2].x, acc[16 * ch + 4 * q + 2].y),
+                                                   pack_bf16x2(acc[16 * ch + 4 * q + 3].x, acc[16 * ch + 4 * q + 3].y));
+                        __syncwarp();
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int rr = 8 * g + sub;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
+                            if (32 * quarter + rr < T.rows_valid)
+                                *reinterpret_cast<uint4*>(ob + (T.out_row0 + 32 * quarter + rr) * a.N + 32 * ch) = v;
+                        }
+                        __syncwarp();
+                    }
                 }
             }
         }
@@ -522,7 +634,7 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
             return FG8_ERR_CUDA;
     } else if (group_mode == FG8_GROUP_K) {
         if (bscale_mode != FG8_BSCALE_ROW128) return FG8_ERR_UNSUPPORTED;
-        if (M_total % 128) return FG8_ERR_INVALID_ARG;
+        if (M_total % 128 || !fg8h::aligned16(sa)) return FG8_ERR_INVALID_ARG;
         if (M_total == 0) return FG8_OK;
         max_tiles = (int64_t)E * (M_total / BM) * nt;
         if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||

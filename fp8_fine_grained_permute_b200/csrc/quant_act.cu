@@ -321,11 +321,13 @@ __global__ void __launch_bounds__(kColThreads) colwise_tiles(ColArgs a) {
     for (int cc = warp; cc < 128; cc += kColThreads / 32) {
         const fg8::QScale q = fg8::make_qscale(s_scale[cc]);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const int row = lane + 32 * g;
-            const uint16_t b = xs[row * kXsStride + cc];
-            const float y = fg8::quot(__uint_as_float((uint32_t)b << 16), q);
-            ts[cc * kTsStride + row] = (uint8_t)(fg8::cvt_e4m3x2(y, 0.0f) & 0xFFu);
+        for (int g = 0; g < 4; g += 2) {
+            const int row = lane + 32 * g;   // and row + 32
+            const float x0 = __uint_as_float((uint32_t)xs[row * kXsStride + cc] << 16);
+            const float x1 = __uint_as_float((uint32_t)xs[(row + 32) * kXsStride + cc] << 16);
+            const uint32_t c = fg8::quant_pair(x0, x1, q);
+            ts[cc * kTsStride + row] = (uint8_t)(c & 0xFFu);
+            ts[cc * kTsStride + row + 32] = (uint8_t)(c >> 8);
         }
     }
     __syncthreads();

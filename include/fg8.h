@@ -159,7 +159,7 @@ fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N
  *            [offsets[e], offsets[e+1]); offsets[E] <= M_total
  *   out      [M_total][N] bf16 or fp32; rows outside [0, offsets[E]) are
  *            not written.  An expert with no rows costs nothing.
- *   N % 128 == 0, K % 128 == 0.
+ *   N % 128 == 0, K % 128 == 0, E <= 1024.
  *
  * group_mode = FG8_GROUP_K (weight gradient; variable contraction per expert):
  *   a        E4M3 [M_total][K], sa fp32 [K/128][M_total]
@@ -168,7 +168,8 @@ fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N
  *            (fg8_quantize_act COLWISE's offsets_out; K = its capacity P)
  *   out      [E][M_total][N]: out[e] = sum over columns [offsets[e],
  *            offsets[e+1]) of the contraction; an expert with no columns gets
- *            zeros.  M_total % 128 == 0, N % 128 == 0, K % 128 == 0.
+ *            zeros.  M_total % 128 == 0, N % 128 == 0, K % 128 == 0, E <= 1024;
+ *            sa and sb 16-byte aligned (the scale vectors are bulk-copied).
  *
  * The fp32 output is the accumulator; the bf16 output is its round-to-
  * nearest-even conversion.  dev_status may be NULL only if no device-side

@@ -106,7 +106,7 @@ def test_quantize_weight_dsv3_full_size_sampled_blocks(oracle):
 
 
 def test_quantize_fast_path_exhaustive_bf16_by_scales(oracle):
-    """Every finite bf16 value x against ~100 tile maxima spanning the bf16 range
+    """Every finite bf16 value x against ~400 tile maxima spanning the bf16 range
     (including subnormal maxima): each row is a 1x128 tile holding its amax and
     127 of the values with |x| <= amax, quantized by the GPU row kernel and by
     the oracle.  Exercises the reciprocal fast path and every fallback."""
@@ -116,7 +116,8 @@ def test_quantize_fast_path_exhaustive_bf16_by_scales(oracle):
     bits = allbits[finite].astype(np.uint16)
     mags = np.abs((bits.astype(np.uint32) << 16).view(np.float32))
     amax_bits = np.unique(np.concatenate([
-        np.linspace(1, 0x7F7F, 90).astype(np.uint16),
+        np.linspace(1, 0x7F7F, 300).astype(np.uint16),
+        np.random.default_rng(12).integers(1, 0x7F80, 100).astype(np.uint16),
         np.array([0x0001, 0x0002, 0x007F, 0x0080, 0x3F80, 0x43E0, 0x7F7F], np.uint16)]))
     rows = []
     for ab in amax_bits:
