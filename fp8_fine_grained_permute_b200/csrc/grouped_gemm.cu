@@ -189,22 +189,6 @@ FG8_DEV void mma_commit(uint32_t bar) {
 FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 lanes x 32 consecutive fp32 columns of TMEM -> 32 registers per thread
-FG8_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 // 32 lanes x 16 consecutive fp32 columns of TMEM -> 16 registers per thread
 FG8_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
@@ -463,14 +447,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (!kGroupK) {
                     const float2 s2 = make_float2(s, s);
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t p[32];
-                        tmem_ld32(taddr + 32 * ch, p);
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float p[16];
+                        tmem_ld16(taddr + 16 * ch, p);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            acc[16 * ch + i] = __ffma2_rn(
-                                make_float2(__uint_as_float(p[2 * i]), __uint_as_float(p[2 * i + 1])),
-                                s2, acc[16 * ch + i]);
+                        for (int i = 0; i < 8; ++i)
+                            acc[8 * ch + i] = __ffma2_rn(make_float2(p[2 * i], p[2 * i + 1]), s2,
+                                                         acc[8 * ch + i]);
                     }
                 } else {
                     // scales of this K block, staged by the producer
@@ -481,20 +464,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const float2 sa2 = make_float2(sa_r, sa_r);
                     const float4* sbv = reinterpret_cast<const float4*>(slot + BM + 128 * half);
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t p[32];
-                        tmem_ld32(taddr + 32 * ch, p);
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float p[16];
+                        tmem_ld16(taddr + 16 * ch, p);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 c4 = col_ok ? sbv[8 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 c4 = col_ok ? sbv[4 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
                             const float2 w0 = __fmul2_rn(make_float2(c4.x, c4.y), sa2);
                             const float2 w1 = __fmul2_rn(make_float2(c4.z, c4.w), sa2);
-                            acc[16 * ch + 2 * i] = __ffma2_rn(
-                                make_float2(__uint_as_float(p[4 * i]), __uint_as_float(p[4 * i + 1])), w0,
-                                acc[16 * ch + 2 * i]);
-                            acc[16 * ch + 2 * i + 1] = __ffma2_rn(
-                                make_float2(__uint_as_float(p[4 * i + 2]), __uint_as_float(p[4 * i + 3])), w1,
-                                acc[16 * ch + 2 * i + 1]);
+                            acc[8 * ch + 2 * i] = __ffma2_rn(make_float2(p[4 * i], p[4 * i + 1]), w0,
+                                                             acc[8 * ch + 2 * i]);
+                            acc[8 * ch + 2 * i + 1] = __ffma2_rn(make_float2(p[4 * i + 2], p[4 * i + 3]),
+                                                                 w1, acc[8 * ch + 2 * i + 1]);
                         }
                     }
                 }
