@@ -18,6 +18,8 @@
 //  * colwise_tiles (weight-gradient operands): 128 tokens x 128 columns per
 //    CTA, amax per column over the tile's tokens, codes written transposed so
 //    that the token axis is contiguous.
+#include <atomic>
+
 #include "fg8_common.cuh"
 
 namespace {
@@ -456,4 +458,59 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
         return fg8h::launch_status();
     }
     return FG8_ERR_INVALID_ARG;
+}
+
+// --------------------------------------------------------------------------
+// permuting mode without a caller-provided workspace
+// --------------------------------------------------------------------------
+//
+// Some callers have no way to allocate device memory: a plugin interface of a
+// host framework that owns every device allocation and hands a kernel only its
+// inputs and outputs, or a latency-critical path that must never enter the
+// allocator.  For them the permuting mode can use a scratch area that lives in
+// the library itself: a file-scope __device__ array, which every GPU that
+// loads libfg8 holds until the process exits.  It is sized for up to
+// kNoAllocMaxExperts experts; larger E is rejected.
+//
+// Host code cannot use the array's name as a device address (it is a host-side
+// stand-in), so on the first call on each device, with that device current,
+// the entry point asks the runtime for the array's device address and caches
+// it.  That first call should therefore come before any stream capture.
+
+namespace {
+
+constexpr int kNoAllocMaxExperts = 256;
+constexpr size_t kNoAllocScratchBytes =
+    256 + 4 * (size_t)kNoAllocMaxExperts + (size_t)kMaxGrid * kNoAllocMaxExperts * 4;  // ~1 MiB
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+
+}  // namespace
+
+extern "C" fg8_status fg8_quantize_act_noalloc(const uint16_t* x, int64_t T, int64_t K,
+                                               const int32_t* topk_ids, int k, int E,
+                                               uint8_t* xq, float* sa, int32_t* row_token,
+                                               int32_t* token_row, int32_t* offsets_out,
+                                               int32_t* dev_status, fg8_stream_t stream) {
+    if (E < 1) return FG8_ERR_INVALID_ARG;
+    if (E > kNoAllocMaxExperts) return FG8_ERR_UNSUPPORTED;
+    size_t off_tot, off_chk;
+    const size_t need = ws_layout(E, &off_tot, &off_chk);
+    if (need > kNoAllocScratchBytes) return FG8_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FG8_ERR_CUDA;
+    void* scratch = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (scratch == nullptr) {
+        if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr)
+            return FG8_ERR_CUDA;
+        g_noalloc_addr[dev].store(scratch, std::memory_order_release);
+    }
+    // the permuting entry point clears the barrier word on every call; the
+    // per-chunk counts and totals are fully written before they are read
+    return fg8_quantize_act(x, T, K, topk_ids, k, E, nullptr, FG8_ROWWISE, xq, sa, row_token,
+                            token_row, offsets_out, nullptr, nullptr, scratch,
+                            kNoAllocScratchBytes, dev_status, stream);
 }

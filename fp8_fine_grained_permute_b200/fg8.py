@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
         L.fg8_quantize_act.restype = _I
         L.fg8_quantize_act.argtypes = [_P, _I64, _I64, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _SZ, _P, _P]
+        L.fg8_quantize_act_noalloc.restype = _I
+        L.fg8_quantize_act_noalloc.argtypes = [_P, _I64, _I64, _P, _I, _I, _P, _P, _P, _P, _P,
+                                               _P, _P]
         L.fg8_quantize_act_workspace.restype = _SZ
         L.fg8_quantize_act_workspace.argtypes = [_I64, _I, _I]
         L.fg8_colwise_capacity.restype = _I64
@@ -124,6 +127,16 @@ def fg8_quantize_act(x, T, K, topk_ids, k, E, offsets_in, layout, xq, sa, row_to
                                   _ptr(offsets_out), _ptr(xqT), _ptr(saT), _ptr(workspace),
                                   ws_bytes, _ptr(dev_status), _stream(stream)),
            "fg8_quantize_act")
+
+
+def fg8_quantize_act_noalloc(x, T, K, topk_ids, k, E, xq, sa, row_token, token_row, offsets_out,
+                             dev_status, stream=None):
+    """Permute + 1x128 quantize using the library's built-in scratch (no
+    workspace argument, nothing allocated; E <= 256)."""
+    _check(lib().fg8_quantize_act_noalloc(_ptr(x), T, K, _ptr(topk_ids), k, E, _ptr(xq), _ptr(sa),
+                                          _ptr(row_token), _ptr(token_row), _ptr(offsets_out),
+                                          _ptr(dev_status), _stream(stream)),
+           "fg8_quantize_act_noalloc")
 
 
 def fg8_quantize_act_workspace(T: int, k: int, E: int) -> int:

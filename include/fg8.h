@@ -114,6 +114,31 @@ fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
                             void* workspace, size_t ws_bytes,
                             int32_t* dev_status, fg8_stream_t stream);
 
+/*
+ * fg8_quantize_act_noalloc -- the permuting mode of fg8_quantize_act
+ * (layout FG8_ROWWISE with topk_ids) for callers that cannot allocate device
+ * memory, such as a plugin whose host framework owns every allocation and
+ * passes only inputs and outputs, or a path that must never enter the
+ * allocator.  The pages have no counterpart of this call; it exists for
+ * those callers only.
+ *   Arguments and outputs are those of fg8_quantize_act in the permuting
+ *   mode, without the workspace.  The scratch the kernel needs is a ~1 MiB
+ *   array inside libfg8 itself (a __device__ variable, so every GPU that
+ *   loads the library holds it until the process exits); the call allocates
+ *   nothing and calls no allocating routine.
+ *   Limit: E <= 256; a larger E returns FG8_ERR_UNSUPPORTED.
+ *   The first call on each device (with that device current) looks up the
+ *   array's device address once; make that first call before any stream
+ *   capture.  All calls on a device share the array: calls that overlap on
+ *   the GPU race with each other.  The library resets what must start at zero
+ *   on every call.
+ */
+fg8_status fg8_quantize_act_noalloc(const uint16_t* x, int64_t T, int64_t K,
+                                    const int32_t* topk_ids, int k, int E,
+                                    uint8_t* xq, float* sa, int32_t* row_token,
+                                    int32_t* token_row, int32_t* offsets_out,
+                                    int32_t* dev_status, fg8_stream_t stream);
+
 /* Workspace bytes needed by fg8_quantize_act in the permuting mode. */
 size_t fg8_quantize_act_workspace(int64_t T, int k, int E);
 
