@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/fg8.h"
@@ -232,5 +233,12 @@ inline fg8_status launch_status() {
 }
 
 int num_sms();  // multiprocessor count of the current device (cached per device)
+
+// 2-D tiled tensor map over a row-major matrix [rows][cols] of `elem_bytes`
+// elements (row stride = cols * elem_bytes), box [box_rows][box_cols].
+// Returns false if the driver entry point is unavailable or rejects the map.
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes,
+                        const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                        uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
 }  // namespace fg8h

@@ -32,8 +32,11 @@
 #include <cuda.h>
 
 #include "fg8_common.cuh"
+#include "fg8_tma.cuh"
 
 namespace {
+
+using namespace fg8::tma;
 
 constexpr int BM = 128, BN = 256, BK = 128;
 constexpr int kStages = 4;
@@ -43,6 +46,17 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr int kEpiWarps = 8;                       // two promotion warpgroups
 constexpr int kCtrlWarps = 4;                      // warpgroup 0: TMA, MMA, 2 idle warps
 constexpr int kThreads = 32 * (kCtrlWarps + kEpiWarps);   // 384
+// Register split (setmaxnreg): the control warpgroup gives registers back and
+// the promotion warpgroups take them, so each promotion thread can hold its
+// 128 accumulators and 64 partial sums in flight.  The split must not exceed
+// what the CTA was launched with (threads x registers per thread), or the
+// increase would wait forever: 128 x 40 + 256 x 232 = 64512 = 384 x 168.  The
+// host refuses to launch unless the compiled kernel has >= kLaunchRegs.
+constexpr int kCtrlRegs = 40;
+constexpr int kEpiRegs = 232;
+constexpr int kLaunchRegs = 168;
+static_assert(32 * kCtrlWarps * kCtrlRegs + 32 * kEpiWarps * kEpiRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;                // two partial buffers of BN columns
 
@@ -90,73 +104,6 @@ struct GemmArgs {
 // PTX wrappers
 // ---------------------------------------------------------------------------
 
-FG8_DEV uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-FG8_DEV void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-FG8_DEV void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-FG8_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-FG8_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n"
-        ".reg .pred p;\n"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        "selp.u32 %0, 1, 0, p;\n"
-        "}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for the phase `parity` of `bar`.  Gives up when another role
-// has aborted or after kWaitLimitNs (then records FG8_ERR_TIMEOUT and raises
-// the CTA's abort flag).
-FG8_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                       int32_t* status) {
-#pragma unroll 1
-    for (int i = 0; i < 256; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = fg8::globaltimer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (fg8::globaltimer_ns() - t0 > fg8::kWaitLimitNs) {
-            fg8::set_status(status, FG8_ERR_TIMEOUT);
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
-
-FG8_DEV void tma_load_2d(const CUtensorMap* map, uint32_t dst, uint32_t bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
-// 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0)
-FG8_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
 // K-major operand tile in shared memory, 128-byte rows, 128-byte swizzle:
 // 8-row atoms 1024 bytes apart (stride byte offset), descriptor version 1.
 FG8_DEV uint64_t smem_desc(uint32_t addr) {
@@ -189,19 +136,30 @@ FG8_DEV void mma_commit(uint32_t bar) {
 FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 lanes x 16 consecutive fp32 columns of TMEM -> 16 registers per thread
-FG8_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
+// 32 lanes x 64 consecutive fp32 columns of TMEM -> 64 registers per thread,
+// waited for inside the same asm statement (the outputs exist only after
+// tcgen05.wait::ld, so no use can be scheduled before the wait).
+FG8_DEV void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+          "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
 }
 
 FG8_DEV uint32_t pack_bf16x2(float lo, float hi) {
@@ -320,7 +278,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint32_t tmem_base = *tmem_slot;
     const int total = s_tiles[a.E];
 
-    if (warp == 0) {
+    if (warp < kCtrlWarps) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+      if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
             uint32_t stage = 0, phase = 0, sc = 0;
@@ -398,7 +358,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             while (!mbar_try_wait(drain_bar, 0) && fg8::globaltimer_ns() - t0 < 100000000ull) {
             }
         }
-    } else if (warp >= kCtrlWarps) {
+      }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
         // ---------------------------------------------------- promotion + epilogue
         const int ep = warp - kCtrlWarps;
         const int half = ep >> 2;            // 128-column half of the tile
@@ -447,13 +409,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (!kGroupK) {
                     const float2 s2 = make_float2(s, s);
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        float p[16];
-                        tmem_ld16(taddr + 16 * ch, p);
+                    for (int ch = 0; ch < 2; ++ch) {
+                        uint32_t p[64];
+                        tmem_ld64(taddr + 64 * ch, p);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            acc[8 * ch + i] = __ffma2_rn(make_float2(p[2 * i], p[2 * i + 1]), s2,
-                                                         acc[8 * ch + i]);
+                        for (int i = 0; i < 32; ++i)
+                            acc[32 * ch + i] = __ffma2_rn(
+                                make_float2(__uint_as_float(p[2 * i]), __uint_as_float(p[2 * i + 1])),
+                                s2, acc[32 * ch + i]);
                     }
                 } else {
                     // scales of this K block, staged by the producer
@@ -464,18 +427,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const float2 sa2 = make_float2(sa_r, sa_r);
                     const float4* sbv = reinterpret_cast<const float4*>(slot + BM + 128 * half);
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        float p[16];
-                        tmem_ld16(taddr + 16 * ch, p);
+                    for (int ch = 0; ch < 2; ++ch) {
+                        uint32_t p[64];
+                        tmem_ld64(taddr + 64 * ch, p);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 c4 = col_ok ? sbv[4 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int i = 0; i < 16; ++i) {
+                            const float4 c4 = col_ok ? sbv[16 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
                             const float2 w0 = __fmul2_rn(make_float2(c4.x, c4.y), sa2);
                             const float2 w1 = __fmul2_rn(make_float2(c4.z, c4.w), sa2);
-                            acc[8 * ch + 2 * i] = __ffma2_rn(make_float2(p[4 * i], p[4 * i + 1]), w0,
-                                                             acc[8 * ch + 2 * i]);
-                            acc[8 * ch + 2 * i + 1] = __ffma2_rn(make_float2(p[4 * i + 2], p[4 * i + 3]),
-                                                                 w1, acc[8 * ch + 2 * i + 1]);
+                            acc[32 * ch + 2 * i] = __ffma2_rn(
+                                make_float2(__uint_as_float(p[4 * i]), __uint_as_float(p[4 * i + 1])), w0,
+                                acc[32 * ch + 2 * i]);
+                            acc[32 * ch + 2 * i + 1] = __ffma2_rn(
+                                make_float2(__uint_as_float(p[4 * i + 2]), __uint_as_float(p[4 * i + 3])), w1,
+                                acc[32 * ch + 2 * i + 1]);
                         }
                     }
                 }
@@ -553,35 +518,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 // host side
 // ---------------------------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 2-D u8 matrix [rows][cols] (row stride = cols bytes), box rows x 128 bytes.
+// 2-D u8 matrix [rows][cols], box rows x 128 bytes, 128-byte swizzle (operand tiles).
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols};
-    cuuint32_t box[2] = {128, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fg8h::make_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, 128,
+                                    box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -627,6 +567,10 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
 
     auto kern = group_mode == FG8_GROUP_K ? grouped_gemm_kernel<true> : grouped_gemm_kernel<false>;
+    // the warpgroup register split must fit in what the CTA is launched with
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, (const void*)kern) != cudaSuccess) return FG8_ERR_CUDA;
+    if (fa.numRegs < kLaunchRegs) return FG8_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return FG8_ERR_CUDA;
