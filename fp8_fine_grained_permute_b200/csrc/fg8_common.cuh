@@ -118,29 +118,62 @@ FG8_DEV uint32_t quant_pair(float x0, float x1, const QScale& q) {
     return cvt_e4m3x2(__fdiv_rn(x0, q.s), __fdiv_rn(x1, q.s));
 }
 
-// Quantize 8 bf16 values (one uint4) with scale context q -> 8 codes (uint2).
-// The fast-path check is made once for all 8 codes, so the rare exact path
-// costs one (usually not taken) branch per 8 elements.
-FG8_DEV uint2 quant8(const uint4& v, const QScale& q) {
+// Fast-path codes of 8 bf16 values (one uint4): the codes of x * r(1 - eps)
+// and of x * r(1 + eps).  No branch, so callers can keep many of these in
+// flight and check them together (exact when lo == hi and !q.exact).
+FG8_DEV void quant8_bracket(const uint4& v, const QScale& q, uint2& lo, uint2& hi) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    if (!q.exact) {
-        const uint64_t rl = pack_f32x2(q.r_lo, q.r_lo), rh = pack_f32x2(q.r_hi, q.r_hi);
-        uint32_t lo[4], hi[4];
+    const uint64_t rl = pack_f32x2(q.r_lo, q.r_lo), rh = pack_f32x2(q.r_hi, q.r_hi);
+    uint32_t l[4], h[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint64_t x = pack_f32x2(bf16_lo(w[i]), bf16_hi(w[i]));
-            lo[i] = cvt_e4m3x2(mul_f32x2(x, rl));
-            hi[i] = cvt_e4m3x2(mul_f32x2(x, rh));
-        }
-        const uint2 cl = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
-        const uint2 ch = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
-        if (cl.x == ch.x && cl.y == ch.y) return cl;
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t x = pack_f32x2(bf16_lo(w[i]), bf16_hi(w[i]));
+        l[i] = cvt_e4m3x2(mul_f32x2(x, rl));
+        h[i] = cvt_e4m3x2(mul_f32x2(x, rh));
     }
+    lo = make_uint2(l[0] | (l[1] << 16), l[2] | (l[3] << 16));
+    hi = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+}
+
+FG8_DEV bool bracket_agrees(const uint2& lo, const uint2& hi) {
+    return ((lo.x ^ hi.x) | (lo.y ^ hi.y)) == 0u;
+}
+
+// Exact codes of 8 bf16 values by IEEE division (the slow path).
+FG8_DEV uint2 quant8_exact(const uint4& v, const QScale& q) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         c[i] = cvt_e4m3x2(__fdiv_rn(bf16_lo(w[i]), q.s), __fdiv_rn(bf16_hi(w[i]), q.s));
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// Quantize 8 bf16 values (one uint4) with scale context q -> 8 codes (uint2).
+FG8_DEV uint2 quant8(const uint4& v, const QScale& q) {
+    uint2 lo, hi;
+    quant8_bracket(v, q, lo, hi);
+    if (!q.exact && bracket_agrees(lo, hi)) return lo;
+    return quant8_exact(v, q);
+}
+
+// Quantize N groups of 8 values sharing one scale context: all fast-path
+// codes are formed first (independent work the scheduler can overlap), then
+// one combined check decides whether any group needs the exact path.
+template <int N>
+FG8_DEV void quant8xN(const uint4 (&v)[N], const QScale& q, uint2 (&c)[N]) {
+    uint2 hi[N];
+    bool ok = !q.exact;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        quant8_bracket(v[i], q, c[i], hi[i]);
+        ok &= bracket_agrees(c[i], hi[i]);
+    }
+    if (!ok) {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            if (q.exact || !bracket_agrees(c[i], hi[i])) c[i] = quant8_exact(v[i], q);
+    }
 }
 
 // max |x| over 8 bf16 values: magnitudes of non-NaN floats order like their

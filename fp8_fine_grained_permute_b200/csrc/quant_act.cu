@@ -17,7 +17,7 @@
 //  * quant_rows    (rows already in expert order): the phase-C row loop only.
 //  * colwise_tiles (weight-gradient operands): 128 tokens x 128 columns per
 //    CTA, amax per column over the tile's tokens, codes written transposed so
-//    that the token axis is contiguous.
+//    that the token axis is contiguous (thread = 2 columns x 32 tokens).
 #include <atomic>
 
 #include "fg8_common.cuh"
@@ -76,22 +76,41 @@ __device__ __forceinline__ void quant_row(const uint16_t* __restrict__ src, int6
             ok[u] = (s0 + u < nseg) && (off < K);
             v[u] = ok[u] ? fg8::ld_stream16(src + off) : make_uint4(0u, 0u, 0u, 0u);
         }
+        // amax of the 4 tiles this half-warp holds (independent shuffle chains)
+        float m[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m[u] = fg8::amax8(v[u]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m[u] = fmaxf(m[u], __shfl_xor_sync(kFull, m[u], o));
+        // fast-path codes of all 4 segments first, one combined check
+        float s[4];
+        fg8::QScale q[4];
+        uint2 c[4], h[4];
+        bool fast = true;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            s[u] = fg8::tile_scale(m[u]);
+            q[u] = fg8::make_qscale(s[u]);
+            fg8::quant8_bracket(v[u], q[u], c[u], h[u]);
+            fast &= !q[u].exact && fg8::bracket_agrees(c[u], h[u]);
+        }
+        if (!fast) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (q[u].exact || !fg8::bracket_agrees(c[u], h[u])) c[u] = fg8::quant8_exact(v[u], q[u]);
+        }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             if (s0 + u >= nseg) break;                 // warp-uniform
-            float m = fg8::amax8(v[u]);
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-            const float s = fg8::tile_scale(m);
-            const fg8::QScale q = fg8::make_qscale(s);
-            const uint2 c = fg8::quant8(v[u], q);
             const int64_t off = (int64_t)(s0 + u) * 256 + 8 * lane;
             const int64_t kb = (int64_t)(s0 + u) * 2 + (lane >> 4);
             for (int j = 0; j < nd; ++j) {
                 const int r = __shfl_sync(kFull, my_row, j);
                 if (ok[u] && r >= 0) {
-                    *reinterpret_cast<uint2*>(xq + (int64_t)r * K + off) = c;
-                    if ((lane & 15) == 0) sa[kb * R + r] = s;
+                    *reinterpret_cast<uint2*>(xq + (int64_t)r * K + off) = c[u];
+                    if ((lane & 15) == 0) sa[kb * R + r] = s[u];
                 }
             }
         }
@@ -118,7 +137,7 @@ struct RouteArgs {
     int32_t* status;
 };
 
-__global__ void __launch_bounds__(kThreads) route_quant(RouteArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
     __shared__ int32_t s_cnt[kMaxE];
     __shared__ int32_t s_off[kMaxE + 1];
     __shared__ int32_t s_warp[33];
@@ -205,7 +224,7 @@ __global__ void __launch_bounds__(kThreads) route_quant(RouteArgs a) {
 // identity mode
 // --------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 quant_rows(const uint16_t* __restrict__ x, int64_t R, int64_t K, uint8_t* __restrict__ xq,
            float* __restrict__ sa) {
     const int lane = threadIdx.x & 31;
@@ -220,19 +239,6 @@ quant_rows(const uint16_t* __restrict__ x, int64_t R, int64_t K, uint8_t* __rest
 // --------------------------------------------------------------------------
 
 constexpr int kColThreads = 256;
-constexpr int kXsStride = 130;   // bf16 per shared row (128 + 2): conflict-free column reads
-constexpr int kTsStride = 144;   // bytes per staged code row (128 + 16), rows 16-byte aligned
-// shared-memory map of colwise_tiles (byte offsets; ts rows are read as 16-byte vectors)
-constexpr size_t kOffTs = 0;
-constexpr size_t kOffXs = kOffTs + 128 * kTsStride;                        // 18432
-constexpr size_t kOffScale = kOffXs + sizeof(uint16_t) * 128 * kXsStride;  // 51712
-constexpr size_t kOffNtile = kOffScale + sizeof(float) * 128;
-constexpr size_t kOffPref = kOffNtile + sizeof(int32_t) * kMaxE;
-constexpr size_t kOffWarp = kOffPref + sizeof(int32_t) * (kMaxE + 4);
-constexpr size_t kColSmem = kOffWarp + sizeof(int32_t) * 36;
-static_assert(kOffTs % 16 == 0 && kTsStride % 16 == 0, "ts rows are read as 16-byte vectors");
-static_assert(kOffXs % 4 == 0 && (kXsStride * 2) % 4 == 0, "xs rows are written as words");
-static_assert(kOffScale % 4 == 0 && kOffNtile % 4 == 0 && kOffWarp % 4 == 0, "word arrays");
 
 struct ColArgs {
     const uint16_t* x;
@@ -248,24 +254,27 @@ struct ColArgs {
     int32_t* padoff_out;
 };
 
+// One CTA per (128-token tile of one expert) x (128 columns).  Thread t owns
+// the column pair p = t % 64 (columns 2p, 2p+1) for the 32 tokens of quarter
+// q = t / 64: it loads them as 32-bit words (a warp load is one 128-byte row
+// piece), reduces its two column maxima in registers (16-bit SIMD max), and
+// the four quarters of a pair combine through shared memory.  Codes are then
+// formed per column on 8 consecutive tokens at a time (bracketed fast path)
+// and stored transposed: 32 contiguous bytes of each column per thread.
 __global__ void __launch_bounds__(kColThreads) colwise_tiles(ColArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t* ts = smem + kOffTs;                                       // [128][kTsStride] codes
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kOffXs);        // [128][kXsStride] bf16
-    float* s_scale = reinterpret_cast<float*>(smem + kOffScale);      // [128]
-    int32_t* s_ntile = reinterpret_cast<int32_t*>(smem + kOffNtile);  // [kMaxE]
-    int32_t* s_pref = reinterpret_cast<int32_t*>(smem + kOffPref);    // [kMaxE + 1]
-    int32_t* s_warp = reinterpret_cast<int32_t*>(smem + kOffWarp);    // [33]
+    __shared__ int32_t s_pref[kMaxE + 1];
+    __shared__ int32_t s_warp[33];
+    __shared__ int32_t s_rows[128];
+    __shared__ uint32_t s_amax[4][64];
 
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int t = threadIdx.x;
     const int E = a.E;
-
     for (int e = t; e < E; e += kColThreads) {
         const int32_t Te = max(0, a.offsets[e + 1] - a.offsets[e]);
-        s_ntile[e] = (Te + 127) / 128;
+        s_pref[e] = (Te + 127) / 128;
     }
     __syncthreads();
-    fg8::block_exclusive_scan(s_ntile, s_pref, E, s_warp);
+    fg8::block_exclusive_scan(s_pref, s_pref, E, s_warp);
     if (blockIdx.x == 0 && blockIdx.y == 0)
         for (int e = t; e <= E; e += kColThreads) a.padoff_out[e] = 128 * s_pref[e];
 
@@ -278,72 +287,64 @@ __global__ void __launch_bounds__(kColThreads) colwise_tiles(ColArgs a) {
     }
     const int e = lo;
     const int tb = tile - s_pref[e];
+    const int64_t pcol = (int64_t)128 * s_pref[e] + 128 * tb;   // padded token column
+    if (pcol + 128 > a.P) return;   // offsets inconsistent with R: never write past the buffers
     const int32_t Te = a.offsets[e + 1] - a.offsets[e];
     const int n_in = min(128, Te - 128 * tb);
     const int64_t row0 = (int64_t)a.offsets[e] + 128 * tb;
     const int64_t col0 = (int64_t)blockIdx.y * 128;
 
-    // load 128 rows x 128 columns (bf16) into shared memory, zeros past n_in
-    {
-        const int ch = t & 15, rr = t >> 4;
-        uint4 v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int row = rr + 16 * i;
-            v[i] = make_uint4(0u, 0u, 0u, 0u);
-            const int64_t lr = row0 + row;
-            if (row < n_in && lr < a.R) {
-                const int64_t sr = a.row_map ? (int64_t)a.row_map[lr] : lr;
-                if (sr >= 0 && sr < a.T_src) v[i] = fg8::ld_stream16(a.x + sr * a.C + col0 + ch * 8);
-            }
+    // source rows of the tile's 128 tokens (-1: padding or out of range)
+    if (t < 128) {
+        const int64_t lr = row0 + t;
+        int32_t sr = -1;
+        if (t < n_in && lr < a.R) {
+            const int64_t v = a.row_map ? (int64_t)a.row_map[lr] : lr;
+            if (v >= 0 && v < a.T_src) sr = (int32_t)v;
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t* d = reinterpret_cast<uint32_t*>(xs + (rr + 16 * i) * kXsStride + ch * 8);
-            d[0] = v[i].x; d[1] = v[i].y; d[2] = v[i].z; d[3] = v[i].w;
-        }
+        s_rows[t] = sr;
     }
     __syncthreads();
 
-    // per-column amax over the tile's rows (padding rows are zero)
-    for (int cc = warp; cc < 128; cc += kColThreads / 32) {
-        float m = 0.0f;
+    const int p = t & 63, q = t >> 6;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(a.x + col0) + p;
+    const int64_t wstride = a.C / 2;    // 32-bit words per source row
+    uint32_t w[32];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const uint16_t b = xs[(lane + 32 * g) * kXsStride + cc];
-            m = fmaxf(m, fabsf(__uint_as_float((uint32_t)b << 16)));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        if (lane == 0) s_scale[cc] = fg8::tile_scale(m);
+    for (int i = 0; i < 32; ++i) {
+        const int32_t sr = s_rows[32 * q + i];
+        w[i] = sr >= 0 ? __ldg(src + (int64_t)sr * wstride) : 0u;
     }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    s_amax[q][p] = m;
     __syncthreads();
+    m = __vmaxu2(__vmaxu2(s_amax[0][p], s_amax[1][p]), __vmaxu2(s_amax[2][p], s_amax[3][p]));
+    const float s0 = fg8::tile_scale(__uint_as_float((m & 0xFFFFu) << 16));   // column 2p
+    const float s1 = fg8::tile_scale(__uint_as_float(m & 0xFFFF0000u));       // column 2p + 1
+    const fg8::QScale q0 = fg8::make_qscale(s0), q1 = fg8::make_qscale(s1);
 
-    // quantize into the transposed staging tile: ts[column][token]
-    for (int cc = warp; cc < 128; cc += kColThreads / 32) {
-        const fg8::QScale q = fg8::make_qscale(s_scale[cc]);
+    // per column: 4 groups of 8 consecutive tokens, bf16 pairs regrouped by column
+    uint4 v0[4], v1[4];
 #pragma unroll
-        for (int g = 0; g < 4; g += 2) {
-            const int row = lane + 32 * g;   // and row + 32
-            const float x0 = __uint_as_float((uint32_t)xs[row * kXsStride + cc] << 16);
-            const float x1 = __uint_as_float((uint32_t)xs[(row + 32) * kXsStride + cc] << 16);
-            const uint32_t c = fg8::quant_pair(x0, x1, q);
-            ts[cc * kTsStride + row] = (uint8_t)(c & 0xFFu);
-            ts[cc * kTsStride + row + 32] = (uint8_t)(c >> 8);
-        }
+    for (int g = 0; g < 4; ++g) {
+        v0[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x5410), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x5410),
+                           __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x5410), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x5410));
+        v1[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x7632), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x7632),
+                           __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x7632), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x7632));
     }
-    __syncthreads();
-
-    const int64_t pcol = (int64_t)128 * s_pref[e] + 128 * tb;   // padded token column
-    if (pcol + 128 > a.P) return;   // offsets inconsistent with R: never write past the buffers
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int idx = t + kColThreads * i;
-        const int cc = idx >> 3, ch = idx & 7;
-        const uint4 v = *reinterpret_cast<const uint4*>(ts + cc * kTsStride + ch * 16);
-        *reinterpret_cast<uint4*>(a.xqT + (col0 + cc) * a.P + pcol + ch * 16) = v;
-    }
-    if (t < 128) a.saT[(pcol / 128) * a.C + col0 + t] = s_scale[t];
+    uint2 c0[4], c1[4];
+    fg8::quant8xN<4>(v0, q0, c0);
+    fg8::quant8xN<4>(v1, q1, c1);
+    uint8_t* d0 = a.xqT + (col0 + 2 * p) * a.P + pcol + 32 * q;
+    uint8_t* d1 = d0 + a.P;
+    reinterpret_cast<uint4*>(d0)[0] = make_uint4(c0[0].x, c0[0].y, c0[1].x, c0[1].y);
+    reinterpret_cast<uint4*>(d0)[1] = make_uint4(c0[2].x, c0[2].y, c0[3].x, c0[3].y);
+    reinterpret_cast<uint4*>(d1)[0] = make_uint4(c1[0].x, c1[0].y, c1[1].x, c1[1].y);
+    reinterpret_cast<uint4*>(d1)[1] = make_uint4(c1[2].x, c1[2].y, c1[3].x, c1[3].y);
+    if (q == 0)
+        reinterpret_cast<float2*>(a.saT + (pcol / 128) * a.C + col0)[p] = make_float2(s0, s1);
 }
 
 size_t ws_layout(int64_t E, size_t* off_totals, size_t* off_chunks) {
@@ -447,14 +448,11 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
         const int64_t P = fg8_colwise_capacity(R, E);
         const int64_t max_tiles = R / 128 + E;
         if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(colwise_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kColSmem) != cudaSuccess)
-            return FG8_ERR_CUDA;
         ColArgs a;
         a.x = x; a.T_src = T; a.R = R; a.C = K; a.row_map = row_token; a.offsets = offsets_in; a.E = E; a.P = P;
         a.xqT = xqT; a.saT = saT; a.padoff_out = offsets_out;
         dim3 grid((unsigned)max_tiles, (unsigned)(K / 128));
-        colwise_tiles<<<grid, kColThreads, kColSmem, st>>>(a);
+        colwise_tiles<<<grid, kColThreads, 0, st>>>(a);
         return fg8h::launch_status();
     }
     return FG8_ERR_INVALID_ARG;
