@@ -41,22 +41,41 @@ FG8_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait for the phase `parity` of `bar`.  Gives up when another role
-// has aborted or after kWaitLimitNs (then records FG8_ERR_TIMEOUT and raises
-// the CTA's abort flag).
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of spinning
+FG8_DEV bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase `parity` of `bar`.  Waiting threads sleep in
+// try_wait (no busy spinning that would take issue slots and shared-memory
+// bandwidth from the warps doing the work); every 16 tries the wait checks
+// whether another role has aborted, and gives up after kWaitLimitNs (then
+// records FG8_ERR_TIMEOUT and raises the CTA's abort flag).
 FG8_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                        int32_t* status) {
-#pragma unroll 1
-    for (int i = 0; i < 256; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = fg8::globaltimer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (fg8::globaltimer_ns() - t0 > fg8::kWaitLimitNs) {
-            fg8::set_status(status, FG8_ERR_TIMEOUT);
-            *abort_flag = 1;
-            return false;
+#pragma unroll 1
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((i & 15) == 0) {
+            if (*abort_flag) return false;
+            if (fg8::globaltimer_ns() - t0 > fg8::kWaitLimitNs) {
+                fg8::set_status(status, FG8_ERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
         }
     }
 }

@@ -39,7 +39,6 @@ namespace {
 using namespace fg8::tma;
 
 constexpr int BM = 128, BN = 256, BK = 128;
-constexpr int kStages = 4;
 constexpr uint32_t kABytes = BM * BK;              // 16 KB
 constexpr uint32_t kBBytes = BN * BK;              // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
@@ -65,28 +64,44 @@ constexpr uint32_t kTmemCols = 512;                // two partial buffers of BN 
 constexpr uint32_t kIdesc =
     (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffStages = 0;
-constexpr uint32_t kOffBars = kStages * kStageBytes;            // 196608
-constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;               // full, empty, tfull, tempty, drain
-constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;          // tmem slot, abort flag
-constexpr uint32_t kOffTiles = kOffMisc + 16;                   // int32 [kMaxE + 1]
-constexpr uint32_t kOffWarp = kOffTiles + 4 * (kMaxE + 4);      // int32 [36]
-// epilogue staging: per promotion warp 32 rows x 16 words (+4 words padding)
+// row-grouped epilogue staging: per promotion warp 32 rows x 16 words (+4 padding)
 constexpr int kStageWords = 20;
 constexpr uint32_t kStagePerWarp = 32 * kStageWords * 4;         // 2560 bytes
-constexpr uint32_t kOffStage = (kOffWarp + 4 * 36 + 15) & ~15u;
+// contraction-grouped epilogue: per promotion warp two 32 x 32 fp32 boxes
+// (4 KB each, 128-byte swizzle) drained by TMA stores
+constexpr uint32_t kBoxBytes = 32 * 32 * 4;
+constexpr uint32_t kTmaStagePerWarp = 2 * kBoxBytes;
 // contraction-grouped mode: per K block the producer also copies the 128 row
-// scales of A and the 256 column scales of B into a ring of kScaleSlots slots.
-// A slot is rewritten kScaleSlots K blocks later, i.e. only after the MMA of
-// K block c+2 has taken the TMEM buffer that the promotion of K block c (the
-// slot's reader) released, so kStages + 2 slots never race.
-constexpr int kScaleSlots = kStages + 2;
+// scales of A and the 256 column scales of B into a ring of slots.  The slot of
+// K block n is rewritten for block n + kScaleSlots.  The producer loads block n
+// only after the MMA of block n - kStages released that stage, and that MMA
+// started only after the promotion of block n - kStages - 2 released its TMEM
+// buffer (having read its scales first).  So kScaleSlots >= kStages + 2 slots
+// are never rewritten before their reader is done.
 constexpr uint32_t kScaleSlotBytes = 4 * (BM + BN);            // 1536
-constexpr uint32_t kOffScales = kOffStage + kEpiWarps * kStagePerWarp;
-constexpr uint32_t kSmemBytes = kOffScales + kScaleSlots * kScaleSlotBytes + 1024;  // + alignment slack
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-static_assert((kStageWords * 4) % 16 == 0 && kOffStage % 16 == 0, "staged rows are 16-byte vectors");
+
+constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+// shared memory map (offsets from a 1024-byte aligned base), per mode
+template <bool kGroupK>
+struct Layout {
+    static constexpr int kStages = kGroupK ? 3 : 4;    // short K loops need fewer
+    static constexpr int kScaleSlots = kStages + 2;
+    static constexpr uint32_t kOffStages = 0;
+    static constexpr uint32_t kOffBars = kStages * kStageBytes;
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;   // full, empty, tfull, tempty, drain
+    static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;   // tmem slot, abort flag
+    static constexpr uint32_t kOffTiles = kOffMisc + 16;            // int32 [kMaxE + 1]
+    static constexpr uint32_t kOffWarp = kOffTiles + 4 * (kMaxE + 4);   // int32 [36]
+    static constexpr uint32_t kOffStage = align_up(kOffWarp + 4 * 36, kGroupK ? 1024 : 16);
+    static constexpr uint32_t kStageAll =
+        kEpiWarps * (kGroupK ? kTmaStagePerWarp : kStagePerWarp);
+    static constexpr uint32_t kOffScales = kOffStage + kStageAll;
+    static constexpr uint32_t kSmemBytes =
+        kOffScales + (kGroupK ? kScaleSlots * kScaleSlotBytes : 0) + 1024;   // + alignment slack
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kOffStage % 16 == 0 && (kStageWords * 4) % 16 == 0, "16-byte staging");
+};
 
 struct GemmArgs {
     const float* sa;
@@ -135,6 +150,24 @@ FG8_DEV void mma_commit(uint32_t bar) {
 
 FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns of TMEM -> 32 registers per thread
+// (waited for inside the same asm statement)
+FG8_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
 
 // 32 lanes x 64 consecutive fp32 columns of TMEM -> 64 registers per thread,
 // waited for inside the same asm statement (the outputs exist only after
@@ -223,7 +256,14 @@ FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const GemmArgs& a, in
 template <bool kGroupK>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs a) {
+    using L = Layout<kGroupK>;
+    constexpr int kStages = L::kStages;
+    constexpr int kScaleSlots = L::kScaleSlots;
+    constexpr uint32_t kOffStages = L::kOffStages, kOffBars = L::kOffBars, kOffMisc = L::kOffMisc;
+    constexpr uint32_t kOffTiles = L::kOffTiles, kOffWarp = L::kOffWarp, kOffStage = L::kOffStage;
+    constexpr uint32_t kOffScales = L::kOffScales;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -368,6 +408,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int r = 32 * quarter + lane;   // tile row owned by this thread
         const int NB = a.N / 128, KBt = a.K / BK;
         uint32_t buf = 0, bphase = 0, sc = 0;
+        uint32_t nbox = 0;    // TMA-store boxes issued by this warp (contraction-grouped)
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
             const Tile T = decode_tile(tile, s_tiles, a, nt);
@@ -426,21 +467,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const float sa_r = slot[r];
                     const float2 sa2 = make_float2(sa_r, sa_r);
                     const float4* sbv = reinterpret_cast<const float4*>(slot + BM + 128 * half);
+                    // per 64 columns: one TMEM load; the first 16 columns' scale vectors
+                    // are read before it (their latency overlaps the load), the
+                    // others 4 vectors (16 columns) at a time just before use
 #pragma unroll
                     for (int ch = 0; ch < 2; ++ch) {
+                        float4 cv[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            cv[i] = col_ok ? sbv[16 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
                         uint32_t p[64];
                         tmem_ld64(taddr + 64 * ch, p);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float4 c4 = col_ok ? sbv[16 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                            const float2 w0 = __fmul2_rn(make_float2(c4.x, c4.y), sa2);
-                            const float2 w1 = __fmul2_rn(make_float2(c4.z, c4.w), sa2);
-                            acc[32 * ch + 2 * i] = __ffma2_rn(
-                                make_float2(__uint_as_float(p[4 * i]), __uint_as_float(p[4 * i + 1])), w0,
-                                acc[32 * ch + 2 * i]);
-                            acc[32 * ch + 2 * i + 1] = __ffma2_rn(
-                                make_float2(__uint_as_float(p[4 * i + 2]), __uint_as_float(p[4 * i + 3])), w1,
-                                acc[32 * ch + 2 * i + 1]);
+                        for (int g = 0; g < 4; ++g) {
+                            if (g > 0) {
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    cv[i] = col_ok ? sbv[16 * ch + 4 * g + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int c = 16 * g + 4 * i;     // column within the 64
+                                const float2 w0 = __fmul2_rn(make_float2(cv[i].x, cv[i].y), sa2);
+                                const float2 w1 = __fmul2_rn(make_float2(cv[i].z, cv[i].w), sa2);
+                                acc[32 * ch + c / 2] = __ffma2_rn(
+                                    make_float2(__uint_as_float(p[c]), __uint_as_float(p[c + 1])), w0,
+                                    acc[32 * ch + c / 2]);
+                                acc[32 * ch + c / 2 + 1] = __ffma2_rn(
+                                    make_float2(__uint_as_float(p[c + 2]), __uint_as_float(p[c + 3])), w1,
+                                    acc[32 * ch + c / 2 + 1]);
+                            }
                         }
                     }
                 }
@@ -451,10 +507,39 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (buf == 0) bphase ^= 1u;
             }
             if (!ok) break;
+            if (kGroupK) {
+                // Epilogue (contraction-grouped, fp32, full 128-row tiles): each
+                // warp writes its 32 rows x 128 columns as four 32 x 32 boxes
+                // through two 4 KB staging buffers (128-byte swizzle: chunk c of
+                // row r sits at chunk c ^ (r & 7), so the row writes are
+                // conflict-free) and TMA-stores them; the stores drain while the
+                // warp moves on to the next tile's promotion.
+                if (col_ok) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t b = (uint32_t)(nbox & 1);
+                        if (lane == 0 && nbox >= 2) bulk_wait_read<1>();   // buffer b drained
+                        __syncwarp();
+                        uint8_t* buf = smem + kOffStage + ep * kTmaStagePerWarp + b * kBoxBytes;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<float4*>(buf + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                                make_float4(acc[16 * j + 2 * c].x, acc[16 * j + 2 * c].y,
+                                            acc[16 * j + 2 * c + 1].x, acc[16 * j + 2 * c + 1].y);
+                        fence_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmOut, smem_u32(buf), col0 + 32 * j,
+                                         (int)(T.out_row0 + 32 * quarter));
+                            bulk_commit();
+                        }
+                        ++nbox;
+                    }
+                }
+            } else if (col_ok) {
             // Epilogue: 16 words of each row at a time go through this warp's
             // staging rows, then every store instruction writes 8 rows x 64
             // contiguous bytes (whole sectors) instead of 32 scattered pieces.
-            if (col_ok) {
                 uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kOffStage) + ep * 32 * kStageWords;
                 uint4* my_row = reinterpret_cast<uint4*>(stg + lane * kStageWords);
                 const int sub = ((lane >> 2) & 1) * 4 + (lane >> 3);  // rows g*8+sub, conflict-free
@@ -502,6 +587,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
             }
         }
+        // TMA stores read shared memory asynchronously: let them finish
+        if (kGroupK && lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -544,7 +631,7 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
 
     const int64_t nt = (N + BN - 1) / BN;
     int64_t max_tiles;
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mOut;
     if (group_mode == FG8_GROUP_M) {
         if (bscale_mode != FG8_BSCALE_BLOCK128) return FG8_ERR_UNSUPPORTED;
         if (M_total == 0) return FG8_OK;
@@ -553,13 +640,19 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
         if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||
             !make_map(&mB, b, (uint64_t)E * N, (uint64_t)K, BN))
             return FG8_ERR_CUDA;
+        mOut = mA;   // unused by the row-grouped epilogue
     } else if (group_mode == FG8_GROUP_K) {
         if (bscale_mode != FG8_BSCALE_ROW128) return FG8_ERR_UNSUPPORTED;
         if (M_total % 128 || !fg8h::aligned16(sa)) return FG8_ERR_INVALID_ARG;
+        if (out_dtype != FG8_OUT_F32) return FG8_ERR_UNSUPPORTED;
         if (M_total == 0) return FG8_OK;
+        if ((int64_t)E * M_total > INT32_MAX) return FG8_ERR_UNSUPPORTED;
         max_tiles = (int64_t)E * (M_total / BM) * nt;
         if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||
-            !make_map(&mB, b, (uint64_t)N, (uint64_t)K, BN))
+            !make_map(&mB, b, (uint64_t)N, (uint64_t)K, BN) ||
+            !fg8h::make_tensor_map_2d(&mOut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out,
+                                      (uint64_t)E * M_total, (uint64_t)N, 32, 32,
+                                      CU_TENSOR_MAP_SWIZZLE_128B))
             return FG8_ERR_CUDA;
     } else {
         return FG8_ERR_INVALID_ARG;
@@ -567,12 +660,14 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
 
     auto kern = group_mode == FG8_GROUP_K ? grouped_gemm_kernel<true> : grouped_gemm_kernel<false>;
+    const uint32_t smem_bytes =
+        group_mode == FG8_GROUP_K ? Layout<true>::kSmemBytes : Layout<false>::kSmemBytes;
     // the warpgroup register split must fit in what the CTA is launched with
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, (const void*)kern) != cudaSuccess) return FG8_ERR_CUDA;
     if (fa.numRegs < kLaunchRegs) return FG8_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes) !=
+        cudaSuccess)
         return FG8_ERR_CUDA;
     GemmArgs args;
     args.sa = sa;
@@ -589,6 +684,6 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     int64_t grid = fg8h::num_sms();
     if (grid > max_tiles) grid = max_tiles;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, kThreads, kSmemBytes, (cudaStream_t)stream>>>(mA, mB, args);
+    kern<<<(unsigned)grid, kThreads, smem_bytes, (cudaStream_t)stream>>>(mA, mB, mOut, args);
     return fg8h::launch_status();
 }

@@ -194,7 +194,9 @@ fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N
  *   out      [E][M_total][N]: out[e] = sum over columns [offsets[e],
  *            offsets[e+1]) of the contraction; an expert with no columns gets
  *            zeros.  M_total % 128 == 0, N % 128 == 0, K % 128 == 0, E <= 1024;
- *            sa and sb 16-byte aligned (the scale vectors are bulk-copied).
+ *            sa and sb 16-byte aligned (the scale vectors are bulk-copied);
+ *            out_dtype must be FG8_OUT_F32 (weight gradients are accumulated
+ *            in fp32; other dtypes return FG8_ERR_UNSUPPORTED).
  *
  * The fp32 output is the accumulator; the bf16 output is its round-to-
  * nearest-even conversion.  dev_status may be NULL only if no device-side
