@@ -150,6 +150,15 @@ class Step:
                                   bytes_colwise(T, K, self.padded_total)),
             "gemm_wgrad": ("tensor", 2 * R * N * K),
         }
+        # bytes each GEMM must move at least: operands read once, output written once
+        # (the weight gradient's fp32 output makes its HBM floor the binding one)
+        self.gemm_bytes = {
+            "gemm_fprop_up": R * K + E * N * K + 2 * R * N,
+            "gemm_dgrad": R * N + E * K * N + 2 * R * K,
+            "gemm_wgrad": (N + K) * self.padded_total + 4 * E * N * K,
+        }
+        if I:
+            self.gemm_bytes["gemm_fprop_down"] = R * I + E * K * I + 2 * R * K
         if I:
             w["gemm_fprop_down"] = ("tensor", 2 * R * K * I)
         return w
@@ -459,13 +468,20 @@ def main():
         ms = kern_ms[name]
         if bound == "tensor":
             ach = amount / (ms * 1e-3) / 1e12
-            entry = {"kernel": name, "bound": "tensor", "ms": ms, "achieved": ach,
-                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": ach / fp8_peak}
+            gbytes = st.gemm_bytes[name]
+            t_tensor = amount / (fp8_peak * 1e12)
+            t_hbm = gbytes / (pk["hbm_gbs"] * 1e9)
+            if t_hbm > t_tensor:         # the output/operand traffic is the floor
+                gb = gbytes / (ms * 1e-3) / 1e9
+                entry = {"kernel": name, "bound": "hbm", "ms": ms, "achieved": gb,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gb / pk["hbm_gbs"],
+                         "tflops": ach, "tensor_frac": ach / fp8_peak}
+            else:
+                entry = {"kernel": name, "bound": "tensor", "ms": ms, "achieved": ach,
+                         "peak": fp8_peak, "unit": "TFLOP/s", "frac": ach / fp8_peak}
+            entry["floor_ms"] = 1e3 * max(t_tensor, t_hbm)
             gemm_flops += amount
             gemm_ms += ms
-            if name == "gemm_wgrad":      # fp32 output of E*N*K words is part of its floor
-                out_bytes = cfg.E * cfg.n_up * cfg.hidden * 4
-                entry["hbm_floor_ms"] = out_bytes / (pk["hbm_gbs"] * 1e9) * 1e3
         else:
             ach = amount / (ms * 1e-3) / 1e9
             entry = {"kernel": name, "bound": "hbm", "ms": ms, "achieved": ach,

@@ -253,6 +253,32 @@ FG8_DEV uint32_t ld_acquire_gpu(const uint32_t* p) {
     return v;
 }
 
+// Grid-wide barrier on a zero-initialised global counter, for kernels whose
+// CTAs are all resident (cooperative launch); `target` = CTAs * phase.
+// Returns false (and records FG8_ERR_TIMEOUT) if the wait runs out.
+FG8_DEV bool grid_barrier(uint32_t* counter, uint32_t target, int32_t* status) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(counter, 1u);
+        const uint64_t t0 = globaltimer_ns();
+        int ok = 1;
+        while (ld_acquire_gpu(counter) < target) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                ok = 0;
+                set_status(status, FG8_ERR_TIMEOUT);
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
 }  // namespace fg8
 
 // Host-side helpers shared by the entry points.

@@ -34,31 +34,6 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // shared helpers
 // --------------------------------------------------------------------------
 
-// Grid-wide barrier on a zero-initialised counter; `target` = CTAs * phase.
-// Returns false (and records FG8_ERR_TIMEOUT) if the wait runs out.
-__device__ bool grid_barrier(uint32_t* counter, uint32_t target, int32_t* status) {
-    __shared__ int s_ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(counter, 1u);
-        const uint64_t t0 = fg8::globaltimer_ns();
-        int ok = 1;
-        while (fg8::ld_acquire_gpu(counter) < target) {
-            if (fg8::globaltimer_ns() - t0 > fg8::kWaitLimitNs) {
-                ok = 0;
-                fg8::set_status(status, FG8_ERR_TIMEOUT);
-                break;
-            }
-            __nanosleep(32);
-        }
-        __threadfence();
-        s_ok = ok;
-    }
-    __syncthreads();
-    return s_ok != 0;
-}
-
 // Quantize one token row (K bf16, K % 128 == 0) in 1x128 tiles and store the
 // codes into the `nd` rows held by lanes 0..nd-1 of `my_row` (negative rows
 // are skipped).  The warp walks the row in 256-element segments: lane l holds
@@ -161,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
     }
     __syncthreads();
     for (int e = t; e < E; e += kThreads) a.chunk_counts[(int64_t)c * E + e] = s_cnt[e];
-    if (!grid_barrier(a.bar, (uint32_t)G, a.status)) return;
+    if (!fg8::grid_barrier(a.bar, (uint32_t)G, a.status)) return;
 
     // ---- phase B: per expert, exclusive scan over chunks (one warp each)
     for (int e = c * kWarps + warp; e < E; e += G * kWarps) {
@@ -180,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
         }
         if (lane == 0) a.totals[e] = carry;
     }
-    if (!grid_barrier(a.bar, 2u * (uint32_t)G, a.status)) return;
+    if (!fg8::grid_barrier(a.bar, 2u * (uint32_t)G, a.status)) return;
 
     // ---- phase C: offsets, stable ranks, index maps
     for (int e = t; e < E; e += kThreads) s_cnt[e] = a.totals[e];

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.fg8_transpose_blockq.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P]
         L.fg8_grouped_gemm.restype = _I
         L.fg8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.fg8_selftest_wait_timeout.restype = _I
+        L.fg8_selftest_wait_timeout.argtypes = [_I, _P, _P, _P]
         L.fg8_status_string.restype = ctypes.c_char_p
         L.fg8_status_string.argtypes = [_I]
         _lib = L
@@ -164,6 +166,11 @@ def fg8_grouped_gemm(a, sa, b, sb, offsets, M_total, N, K, E, group_mode, bscale
                                   N, K, E, group_mode, bscale_mode, out_dtype, _ptr(out),
                                   _ptr(dev_status), _stream(stream)),
            "fg8_grouped_gemm")
+
+
+def fg8_selftest_wait_timeout(which, scratch, dev_status, stream=None):
+    _check(lib().fg8_selftest_wait_timeout(which, _ptr(scratch), _ptr(dev_status), _stream(stream)),
+           "fg8_selftest_wait_timeout")
 
 
 def fg8_status_string(status: int) -> str:

@@ -209,6 +209,19 @@ fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa,
                             int group_mode, int bscale_mode, int out_dtype, void* out,
                             int32_t* dev_status, fg8_stream_t stream);
 
+/*
+ * fg8_selftest_wait_timeout -- diagnostic of the failure-detection path (the
+ * pages have no counterpart).  Runs one of the library's bounded device waits
+ * on a condition that nothing satisfies, so that it runs out after its limit
+ * (about 2 s), writes FG8_ERR_TIMEOUT to *dev_status and returns; the context
+ * stays usable.  Faults nothing.
+ *   which = 0: the grid-wide barrier of the permuting quantizer
+ *              (scratch: one device uint32, cleared by the call)
+ *   which = 1: the mbarrier wait used by the GEMM pipeline (scratch unused)
+ */
+fg8_status fg8_selftest_wait_timeout(int which, uint32_t* scratch, int32_t* dev_status,
+                                     fg8_stream_t stream);
+
 /* Static string naming a status. */
 const char* fg8_status_string(fg8_status s);
 
