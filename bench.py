@@ -87,6 +87,85 @@ def bytes_transpose(E, N, K):
     return 2 * (E * N * K + 4 * E * N * K // 16384)
 
 
+def padded_total_of(cfg: W.MoEConfig) -> int:
+    counts = np.bincount(W.route(cfg).ravel(), minlength=cfg.E)
+    return int(((counts + 127) // 128 * 128).sum())
+
+
+def work_of(cfg: W.MoEConfig, padded_total: int):
+    """Per kernel family of one step: (bound, algorithmic amount) and, for the
+    GEMMs, the bytes they must move at least (operands once, output once)."""
+    T, K, k, E, R, N, I = cfg.T, cfg.hidden, cfg.k, cfg.E, cfg.R, cfg.n_up, cfg.inter
+    w = {
+        "quant_act_permute": ("hbm", bytes_route_quant(T, K, k, E)),
+        "quant_weight": ("hbm", bytes_weight_quant(E, N, K) + (bytes_weight_quant(E, K, I) if I else 0)),
+        "gemm_fprop_up": ("tensor", 2 * R * N * K),
+        "transpose_blockq": ("hbm", bytes_transpose(E, N, K)),
+        "quant_act_rows": ("hbm", bytes_rows_quant(R, N) + (bytes_rows_quant(R, I) if I else 0)),
+        "gemm_dgrad": ("tensor", 2 * R * K * N),
+        "quant_act_colwise": ("hbm", bytes_colwise(R, N, padded_total) + bytes_colwise(T, K, padded_total)),
+        "gemm_wgrad": ("tensor", 2 * R * N * K),
+    }
+    gemm_bytes = {
+        "gemm_fprop_up": R * K + E * N * K + 2 * R * N,
+        "gemm_dgrad": R * N + E * K * N + 2 * R * K,
+        "gemm_wgrad": (N + K) * padded_total + 4 * E * N * K,
+    }
+    if I:
+        w["gemm_fprop_down"] = ("tensor", 2 * R * K * I)
+        gemm_bytes["gemm_fprop_down"] = R * I + E * K * I + 2 * R * K
+    return w, gemm_bytes
+
+
+# DRAM bytes (read + write) per kernel family of one step, from one
+# `ncu --set full` capture of the Kanana-sized step (a few GB on the device;
+# the DeepSeek-V3-shaped step is too large to capture under full sets).  They
+# are scaled to another workload by the ratio of algorithmic bytes, and
+# dropped (traffic: null) when the kernel sources differ from the ones the
+# counters were taken on (short sha1 of the kernel file + shared headers).
+TRAFFIC_CAPTURE = {
+    "config": "kanana",
+    "families": {
+        "quant_act_permute": (228.7e6, "quant_act", "afcb9e785c95"),
+        "quant_weight": (792.6e6, "quant_weight", "5af2cf679f5d"),
+        "gemm_fprop_up": (680.7e6, "gemm", "9ea80bdb42f9"),
+        "gemm_fprop_down": (530.0e6, "gemm", "9ea80bdb42f9"),
+        "transpose_blockq": (348.3e6, "transpose", "c1e4961cfa8c"),
+        "quant_act_rows": (593.2e6, "quant_act", "afcb9e785c95"),
+        "gemm_dgrad": (722.6e6, "gemm", "9ea80bdb42f9"),
+        "quant_act_colwise": (662.3e6, "quant_act", "afcb9e785c95"),
+        "gemm_wgrad": (1152.2e6, "gemm", "9ea80bdb42f9"),
+    },
+}
+_SRC = {"quant_act": ["quant_act.cu"], "quant_weight": ["quant_weight.cu"],
+        "transpose": ["transpose_blockq.cu"], "gemm": ["grouped_gemm.cu", "fg8_tma.cuh"]}
+
+
+def source_hash(group: str) -> str:
+    import hashlib
+    h = hashlib.sha1()
+    base = os.path.join(ROOT, "fp8_fine_grained_permute_b200", "csrc")
+    for f in _SRC[group] + ["fg8_common.cuh"]:
+        with open(os.path.join(base, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(family: str, cfg: W.MoEConfig, padded_total: int):
+    entry = TRAFFIC_CAPTURE["families"].get(family)
+    if entry is None:
+        return None
+    bytes_cap, group, sha = entry
+    if source_hash(group) != sha:
+        return None
+    cap = W.CONFIGS[TRAFFIC_CAPTURE["config"]]
+    w_cap, gb_cap = work_of(cap, padded_total_of(cap))
+    w_now, gb_now = work_of(cfg, padded_total)
+    num = gb_now.get(family, w_now[family][1])
+    den = gb_cap.get(family, w_cap[family][1])
+    return bytes_cap * num / den
+
+
 # --------------------------------------------------------------------------
 # the workload on one GPU
 # --------------------------------------------------------------------------
@@ -134,34 +213,7 @@ class Step:
         self.xT, self.sxT, self.pad_x = e((K, self.P), u8), e((self.P // 128, K), f32), e(E + 1, i32)
         self.dw = e((E, N, K), f32)
         self.launches_per_step = 0
-        self.work = self._work()
-
-    def _work(self):
-        c = self.cfg
-        T, K, k, E, R, N, I = c.T, c.hidden, c.k, c.E, c.R, c.n_up, c.inter
-        w = {
-            "quant_act_permute": ("hbm", bytes_route_quant(T, K, k, E)),
-            "quant_weight": ("hbm", bytes_weight_quant(E, N, K) + (bytes_weight_quant(E, K, I) if I else 0)),
-            "gemm_fprop_up": ("tensor", 2 * R * N * K),
-            "transpose_blockq": ("hbm", bytes_transpose(E, N, K)),
-            "quant_act_rows": ("hbm", bytes_rows_quant(R, N) + (bytes_rows_quant(R, I) if I else 0)),
-            "gemm_dgrad": ("tensor", 2 * R * K * N),
-            "quant_act_colwise": ("hbm", bytes_colwise(R, N, self.padded_total) +
-                                  bytes_colwise(T, K, self.padded_total)),
-            "gemm_wgrad": ("tensor", 2 * R * N * K),
-        }
-        # bytes each GEMM must move at least: operands read once, output written once
-        # (the weight gradient's fp32 output makes its HBM floor the binding one)
-        self.gemm_bytes = {
-            "gemm_fprop_up": R * K + E * N * K + 2 * R * N,
-            "gemm_dgrad": R * N + E * K * N + 2 * R * K,
-            "gemm_wgrad": (N + K) * self.padded_total + 4 * E * N * K,
-        }
-        if I:
-            self.gemm_bytes["gemm_fprop_down"] = R * I + E * K * I + 2 * R * K
-        if I:
-            w["gemm_fprop_down"] = ("tensor", 2 * R * K * I)
-        return w
+        self.work, self.gemm_bytes = work_of(cfg, self.padded_total)
 
     def run(self, stream, marks=None):
         """Launch one step on `stream`.  With `marks`, record an event pair
@@ -489,6 +541,7 @@ def main():
             q_bytes += amount
             q_ms += ms
         entry["share"] = ms / ms_step
+        entry["traffic"] = measured_traffic(name, cfg, st.padded_total)
         kernels.append(entry)
     dom = max(kernels, key=lambda d: d["ms"])
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
@@ -553,7 +606,10 @@ def main():
             "quantize_frac_of_hbm": quant_gbs / world / pk["hbm_gbs"],
             "roofline": {"kernel": dom["kernel"], "bound": dom["bound"], "achieved": dom["achieved"],
                          "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
-                         "traffic": None,
+                         "traffic": measured_traffic(dom["kernel"], cfg, st.padded_total),
+                         "traffic_source": f"ncu --set full DRAM bytes of the {TRAFFIC_CAPTURE['config']} "
+                                           "step, scaled by algorithmic bytes; null if the kernel "
+                                           "changed since",
                          "peak_source": f"{pk['source']}: HBM {pk['hbm_gbs']} GB/s; FP8 = "
                                         f"{FP8_OVER_BF16} x sustained BF16 {pk['bf16_sus']} TFLOP/s"},
             "kernels": kernels,
