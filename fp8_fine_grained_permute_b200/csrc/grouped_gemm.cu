@@ -8,24 +8,33 @@
 // tensor-core instruction (its block-scaled form takes power-of-two scales at
 // 32-element granularity).  Instead each 128-wide K block is multiplied on the
 // tensor core into its own TMEM partial (fp32), and the promotion warps add
-// partial * sA * sB into fp32 accumulators held in registers: the paged
-// design's "CUDA-core promotion", with the partial sums living in TMEM.
+// partial * sA * sB into fp32 accumulators held in registers: DeepSeek-V3's
+// promotion to CUDA cores, with the partial sums living in TMEM.
 //
-// CTA = one persistent worker per SM, 10 warps:
+// CTA = one persistent worker per SM, 12 warps (setmaxnreg gives the control
+// warpgroup 40 registers a thread and the promotion warpgroups 232):
 //   warp 0      TMA producer: A tile 128x128 B and B tile 256x128 B per K block
-//               into a 4-stage ring (48 KB per stage), 128-byte swizzle.
+//               into a 4-stage (row-grouped) or 3-stage (contraction-grouped)
+//               ring of 48 KB stages, 128-byte swizzle; contraction-grouped, it
+//               also bulk-copies the K block's 128 + 256 scales into a slot ring.
 //   warp 1      TMEM allocator + MMA issuer: 4 x tcgen05.mma (M=128, N=256,
 //               K=32, E4M3 x E4M3 -> f32) per K block into one of two TMEM
 //               partial buffers (2 x 256 columns); tcgen05.commit frees the smem
 //               stage and publishes the partial.
-//   warps 2..9  promotion + epilogue: two warpgroups, one per 128-column half;
-//               thread = one output row; tcgen05.ld the partial, release the
-//               buffer, acc = fma(partial, sA*sB, acc); after the last K block
-//               convert and store the row segment.
+//   warps 2, 3  idle.
+//   warps 4..11 promotion + epilogue: two warpgroups, one per 128-column half.
+//               Row-grouped (one scale per row and K block): thread = one output
+//               row, 32x32b loads.  Contraction-grouped (a scale per row and per
+//               column): 16x256b loads, thread = 4 rows x 32 columns, so it reads
+//               16 column-scale pairs instead of 128 scales per K block.
+//               acc = fma(partial, sA*sB, acc), then release the buffer; after
+//               the last K block the tile goes out through shared memory (8-row
+//               x 64-byte stores, or 32x32 fp32 boxes drained by TMA stores).
 // Tiles are 128 rows x 256 columns; the tile list (expert, m-tile, n-tile) is
-// rebuilt on the device from the expert offsets, so offsets never travel to the
-// host.  Zero-row experts have no tiles (row-grouped mode); in the
-// contraction-grouped mode an expert with no tokens writes zeros.
+// rebuilt on the device from the expert offsets (kept in shared memory), so
+// offsets never travel to the host.  Zero-row experts have no tiles
+// (row-grouped mode); in the contraction-grouped mode an expert with no tokens
+// writes zeros.
 //
 // Every mbarrier wait is bounded (FG8_ERR_TIMEOUT in *status, then the roles
 // wind down and TMEM is released); the kernel never traps.
@@ -92,7 +101,8 @@ struct Layout {
     static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;   // full, empty, tfull, tempty, drain
     static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;   // tmem slot, abort flag
     static constexpr uint32_t kOffTiles = kOffMisc + 16;            // int32 [kMaxE + 1]
-    static constexpr uint32_t kOffWarp = kOffTiles + 4 * (kMaxE + 4);   // int32 [36]
+    static constexpr uint32_t kOffOffs = kOffTiles + 4 * (kMaxE + 4);   // int32 [kMaxE + 1]
+    static constexpr uint32_t kOffWarp = kOffOffs + 4 * (kMaxE + 4);    // int32 [36]
     static constexpr uint32_t kOffStage = align_up(kOffWarp + 4 * 36, kGroupK ? 1024 : 16);
     static constexpr uint32_t kStageAll =
         kEpiWarps * (kGroupK ? kTmaStagePerWarp : kStagePerWarp);
@@ -151,24 +161,6 @@ FG8_DEV void mma_commit(uint32_t bar) {
 FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 lanes x 32 consecutive fp32 columns of TMEM -> 32 registers per thread
-// (waited for inside the same asm statement)
-FG8_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-        "tcgen05.wait::ld.sync.aligned;\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
 // 32 lanes x 64 consecutive fp32 columns of TMEM -> 64 registers per thread,
 // waited for inside the same asm statement (the outputs exist only after
 // tcgen05.wait::ld, so no use can be scheduled before the wait).
@@ -195,6 +187,27 @@ FG8_DEV void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
         : "memory");
 }
 
+// Two 16-lane halves' worth of the 16x256b shape, 8 repetitions: thread t of
+// the warp gets, for repetition j, the fp32 values at (lane t/4, column
+// 8j + 2(t%4) + {0,1}) in r[4j], r[4j+1] and at (lane t/4 + 8, same columns)
+// in r[4j+2], r[4j+3], lanes counted from the address's lane field.  Waited
+// for inside the statement.
+FG8_DEV void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
 FG8_DEV uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -216,18 +229,27 @@ struct Tile {
     int64_t out_row0;   // first output row
 };
 
-FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const GemmArgs& a, int nt) {
-    int lo = 0, hi = a.E;   // largest e with s_tiles[e] <= tile
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (s_tiles[mid] <= tile) lo = mid; else hi = mid;
+// s_tiles: exclusive prefix of tiles per expert (E + 1 entries), s_off: the
+// expert offsets, both in shared memory.  A thread's tiles only increase, so
+// the expert of its previous tile (e_hint) starts the search.
+FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const int32_t* s_off, const GemmArgs& a,
+                         int nt, int& e_hint) {
+    int lo = e_hint;   // s_tiles[lo] <= tile; find the largest such e
+    if (s_tiles[lo + 1] <= tile) {
+        int hi = a.E;  // s_tiles[E] = total > tile
+        ++lo;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_tiles[mid] <= tile) lo = mid; else hi = mid;
+        }
     }
+    e_hint = lo;
     Tile T;
     T.e = lo;
     const int local = tile - s_tiles[lo];
     const int mt = local / nt, ntile = local - mt * nt;
     T.n0 = ntile * BN;
-    const int32_t o0 = a.offsets[lo], o1 = a.offsets[lo + 1];
+    const int32_t o0 = s_off[lo], o1 = s_off[lo + 1];
     if (a.mode == FG8_GROUP_M) {
         T.rowA = (int64_t)o0 + (int64_t)mt * BM;
         // rows past M_total (offsets inconsistent with the buffers) are never touched
@@ -277,6 +299,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     int32_t* s_tiles = reinterpret_cast<int32_t*>(smem + kOffTiles);
+    int32_t* s_off = reinterpret_cast<int32_t*>(smem + L::kOffOffs);
     int32_t* s_warp = reinterpret_cast<int32_t*>(smem + kOffWarp);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -310,6 +333,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                                 : (int32_t)(a.M_total / BM);
         s_tiles[e] = cnt * nt;
     }
+    for (int e = threadIdx.x; e <= a.E; e += kThreads) s_off[e] = a.offsets[e];
     __syncthreads();
     fg8::block_exclusive_scan(s_tiles, s_tiles, a.E, s_warp);
     tc_fence_before();
@@ -324,9 +348,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
             uint32_t stage = 0, phase = 0, sc = 0;
+            int e_hint = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile T = decode_tile(tile, s_tiles, a, nt);
+                const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
                 for (int kb = 0; kb < T.nkb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status)) {
                         ok = false;
@@ -366,9 +391,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+            int e_hint = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile T = decode_tile(tile, s_tiles, a, nt);
+                const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
                 for (int kb = 0; kb < T.nkb; ++kb) {
                     if (!mbar_wait(tempty_bar(buf), bphase ^ 1u, abort_flag, a.status) ||
                         !mbar_wait(full_bar(stage), phase, abort_flag, a.status)) {
@@ -405,39 +431,46 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int ep = warp - kCtrlWarps;
         const int half = ep >> 2;            // 128-column half of the tile
         const int quarter = warp & 3;        // TMEM lane quarter this warp may access
-        const int r = 32 * quarter + lane;   // tile row owned by this thread
+        const int r = 32 * quarter + lane;   // tile row owned by this thread (row-grouped)
+        const int g4 = lane >> 2, c2 = 2 * (lane & 3);   // 16x256b position (contraction-grouped)
         const int NB = a.N / 128, KBt = a.K / BK;
         uint32_t buf = 0, bphase = 0, sc = 0;
         uint32_t nbox = 0;    // TMA-store boxes issued by this warp (contraction-grouped)
+        int e_hint = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const Tile T = decode_tile(tile, s_tiles, a, nt);
-            const bool row_ok = r < T.rows_valid;
-            const int col0 = T.n0 + 128 * half;
-            const bool col_ok = col0 < a.N;
             float2 acc[64];   // columns 2i, 2i + 1 of this thread's 128-column half
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            const int kb0 = T.kx0 / BK;
-            // row-grouped mode: scales prefetched two K blocks ahead in registers
-            const float* sa_p = a.sa + T.rowA + r;
-            const float* sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
-            float sa_c = 0.f, sa_n = 0.f, sb_c = 0.f, sb_n = 0.f;
-            if (!kGroupK) {
-                if (row_ok && T.nkb > 0) sa_c = __ldg(sa_p);
-                if (row_ok && T.nkb > 1) sa_n = __ldg(sa_p + a.M_total);
-                if (col_ok && T.nkb > 0) sb_c = __ldg(sb_p);
-                if (col_ok && T.nkb > 1) sb_n = __ldg(sb_p + 1);
+            // Only what the K loop needs stays live through it; the epilogue
+            // decodes the tile again (registers are the promotion's limit).
+            int nkb;
+            bool row_ok, col_ok;
+            const float* sa_p;
+            const float* sb_p;
+            {
+                const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
+                nkb = T.nkb;
+                row_ok = r < T.rows_valid;
+                const int col0 = T.n0 + 128 * half;
+                col_ok = col0 < a.N;
+                sa_p = a.sa + T.rowA + r;
+                sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
             }
-            for (int kb = 0; kb < T.nkb; ++kb) {
+            // row-grouped mode: the scales of the next K block are loaded while
+            // this one is promoted
+            float sa_n = 0.f, sb_n = 0.f;
+            if (!kGroupK) {
+                if (row_ok && nkb > 0) sa_n = __ldg(sa_p);
+                if (col_ok && nkb > 0) sb_n = __ldg(sb_p);
+            }
+            for (int kb = 0; kb < nkb; ++kb) {
                 float s = 0.f;
                 if (!kGroupK) {
-                    s = sa_c * sb_c;
-                    sa_c = sa_n;
-                    sb_c = sb_n;
-                    if (kb + 2 < T.nkb) {
-                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 2) * a.M_total);
-                        if (col_ok) sb_n = __ldg(sb_p + kb + 2);
+                    s = sa_n * sb_n;
+                    if (kb + 1 < nkb) {
+                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 1) * a.M_total);
+                        if (col_ok) sb_n = __ldg(sb_p + kb + 1);
                     }
                 }
                 if (!mbar_wait(tfull_bar(buf), bphase, abort_flag, a.status)) {
@@ -460,42 +493,42 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                                 s2, acc[32 * ch + i]);
                     }
                 } else {
-                    // scales of this K block, staged by the producer
+                    // Both scales vary along the tile here (row scale of A, column
+                    // scale of B), so the partial is read in the 16x256b shape: a
+                    // thread holds 4 rows x 32 columns (rows g4 + 8k, columns
+                    // 8j + c2 + {0,1} of each 64-column group) and needs only 16
+                    // column-scale pairs and 4 row scales per K block, read from the
+                    // producer's slot with distinct addresses instead of 128
+                    // broadcast values.  acc[(cg * 8 + j) * 4 + k] holds row k's pair.
                     const float* slot = reinterpret_cast<const float*>(
                         smem + kOffScales + (sc % kScaleSlots) * kScaleSlotBytes);
                     ++sc;
-                    const float sa_r = slot[r];
-                    const float2 sa2 = make_float2(sa_r, sa_r);
-                    const float4* sbv = reinterpret_cast<const float4*>(slot + BM + 128 * half);
-                    // per 64 columns: one TMEM load; the first 16 columns' scale vectors
-                    // are read before it (their latency overlaps the load), the
-                    // others 4 vectors (16 columns) at a time just before use
+                    float sak[4];
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        float4 cv[4];
+                    for (int k = 0; k < 4; ++k) sak[k] = slot[32 * quarter + g4 + 8 * k];
+                    const float* sbp = slot + BM + 128 * half + c2;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            cv[i] = col_ok ? sbv[16 * ch + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                        uint32_t p[64];
-                        tmem_ld64(taddr + 64 * ch, p);
+                    for (int cg = 0; cg < 2; ++cg) {
+                        float2 sb2[8];
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            if (g > 0) {
+                        for (int j = 0; j < 8; ++j)
+                            sb2[j] = col_ok ? *reinterpret_cast<const float2*>(sbp + 64 * cg + 8 * j)
+                                            : make_float2(0.f, 0.f);
 #pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    cv[i] = col_ok ? sbv[16 * ch + 4 * g + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                            }
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t p[32];
+                            tmem_ld16x256_x8(taddr + ((16u * h) << 16) + 64 * cg, p);
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int c = 16 * g + 4 * i;     // column within the 64
-                                const float2 w0 = __fmul2_rn(make_float2(cv[i].x, cv[i].y), sa2);
-                                const float2 w1 = __fmul2_rn(make_float2(cv[i].z, cv[i].w), sa2);
-                                acc[32 * ch + c / 2] = __ffma2_rn(
-                                    make_float2(__uint_as_float(p[c]), __uint_as_float(p[c + 1])), w0,
-                                    acc[32 * ch + c / 2]);
-                                acc[32 * ch + c / 2 + 1] = __ffma2_rn(
-                                    make_float2(__uint_as_float(p[c + 2]), __uint_as_float(p[c + 3])), w1,
-                                    acc[32 * ch + c / 2 + 1]);
+                            for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                                for (int kk = 0; kk < 2; ++kk) {
+                                    const int k = 2 * h + kk;
+                                    const float2 w = __fmul2_rn(sb2[j], make_float2(sak[k], sak[k]));
+                                    acc[(cg * 8 + j) * 4 + k] = __ffma2_rn(
+                                        make_float2(__uint_as_float(p[4 * j + 2 * kk]),
+                                                    __uint_as_float(p[4 * j + 2 * kk + 1])),
+                                        w, acc[(cg * 8 + j) * 4 + k]);
+                                }
                             }
                         }
                     }
@@ -507,29 +540,39 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (buf == 0) bphase ^= 1u;
             }
             if (!ok) break;
+            const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
+            const int col0 = T.n0 + 128 * half;
             if (kGroupK) {
                 // Epilogue (contraction-grouped, fp32, full 128-row tiles): each
                 // warp writes its 32 rows x 128 columns as four 32 x 32 boxes
-                // through two 4 KB staging buffers (128-byte swizzle: chunk c of
-                // row r sits at chunk c ^ (r & 7), so the row writes are
-                // conflict-free) and TMA-stores them; the stores drain while the
-                // warp moves on to the next tile's promotion.
+                // through two 4 KB staging buffers and TMA-stores them; the stores
+                // drain while the warp moves on to the next tile's promotion.
+                // 128-byte swizzle: 16-byte chunk c of box row rr sits at chunk
+                // c ^ (rr & 7); the four lanes of a row write 32 contiguous bytes,
+                // so each 8-byte store of the warp is two conflict-free wavefronts.
                 if (col_ok) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
+                    for (int bx = 0; bx < 4; ++bx) {
                         const uint32_t b = (uint32_t)(nbox & 1);
                         if (lane == 0 && nbox >= 2) bulk_wait_read<1>();   // buffer b drained
                         __syncwarp();
-                        uint8_t* buf = smem + kOffStage + ep * kTmaStagePerWarp + b * kBoxBytes;
+                        uint8_t* box = smem + kOffStage + ep * kTmaStagePerWarp + b * kBoxBytes;
+                        const int cg = bx >> 1;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<float4*>(buf + lane * 128 + ((c ^ (lane & 7)) * 16)) =
-                                make_float4(acc[16 * j + 2 * c].x, acc[16 * j + 2 * c].y,
-                                            acc[16 * j + 2 * c + 1].x, acc[16 * j + 2 * c + 1].y);
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int j = 4 * (bx & 1) + jj;
+                            const int chunk = 2 * jj + ((lane & 3) >> 1);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int rr = g4 + 8 * k;
+                                *reinterpret_cast<float2*>(box + rr * 128 + ((chunk ^ (rr & 7)) << 4) +
+                                                           8 * (lane & 1)) = acc[(cg * 8 + j) * 4 + k];
+                            }
+                        }
                         fence_async_shared();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_2d(&tmOut, smem_u32(buf), col0 + 32 * j,
+                            tma_store_2d(&tmOut, smem_u32(box), col0 + 32 * bx,
                                          (int)(T.out_row0 + 32 * quarter));
                             bulk_commit();
                         }
