@@ -40,6 +40,8 @@
 // wind down and TMEM is released); the kernel never traps.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "fg8_common.cuh"
 #include "fg8_tma.cuh"
 
@@ -91,6 +93,19 @@ constexpr uint32_t kScaleSlotBytes = 4 * (BM + BN);            // 1536
 
 constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
+// contraction-grouped mode: tiles are handed out at run time.  The producer
+// takes the next tile number from a device counter (zeroed before the launch),
+// decodes it and publishes what the other roles need (K blocks, first output
+// row and column) through a ring of kTileRing shared slots; the MMA thread and
+// the promotion warps read the ring.  Experts with few tokens are output-bound
+// (a 128 KB fp32 tile per 128x256 block) and experts with many are math-bound,
+// so the order interleaves the tiles of kMix experts of different sizes (one
+// from each size quantile) to keep both busy; within an expert, consecutive
+// tiles share their A rows.
+constexpr int kTileRing = 8;
+constexpr int kMix = 4;
+constexpr int kCtrSlots = 64;   // launches that may run at the same time
+
 // shared memory map (offsets from a 1024-byte aligned base), per mode
 template <bool kGroupK>
 struct Layout {
@@ -98,9 +113,13 @@ struct Layout {
     static constexpr int kScaleSlots = kStages + 2;
     static constexpr uint32_t kOffStages = 0;
     static constexpr uint32_t kOffBars = kStages * kStageBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;   // full, empty, tfull, tempty, drain
+    // full, empty, tfull, tempty, drain (+ tile ring full / empty, contraction-grouped)
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kGroupK ? 2 * kTileRing : 0);
     static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;   // tmem slot, abort flag
-    static constexpr uint32_t kOffTiles = kOffMisc + 16;            // int32 [kMaxE + 1]
+    static constexpr uint32_t kOffRing = align_up(kOffMisc + 16, 16);  // int4 [kTileRing]
+    // row-grouped: tiles per expert, exclusive prefix; contraction-grouped:
+    // the experts in processing order
+    static constexpr uint32_t kOffTiles = kOffRing + 16 * kTileRing;   // int32 [kMaxE + 1]
     static constexpr uint32_t kOffOffs = kOffTiles + 4 * (kMaxE + 4);   // int32 [kMaxE + 1]
     static constexpr uint32_t kOffWarp = kOffOffs + 4 * (kMaxE + 4);    // int32 [36]
     static constexpr uint32_t kOffStage = align_up(kOffWarp + 4 * 36, kGroupK ? 1024 : 16);
@@ -123,6 +142,7 @@ struct GemmArgs {
     int out_f32;
     void* out;
     int32_t* status;
+    unsigned int* tile_ctr;   // contraction-grouped: zeroed tile counter
 };
 
 // ---------------------------------------------------------------------------
@@ -229,8 +249,8 @@ struct Tile {
     int64_t out_row0;   // first output row
 };
 
-// s_tiles: exclusive prefix of tiles per expert (E + 1 entries), s_off: the
-// expert offsets, both in shared memory.  A thread's tiles only increase, so
+// Row-grouped: s_tiles is the exclusive prefix of tiles per expert (E + 1
+// entries), s_off the expert offsets, both in shared memory.  A thread's tiles only increase, so
 // the expert of its previous tile (e_hint) starts the search.
 FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const int32_t* s_off, const GemmArgs& a,
                          int nt, int& e_hint) {
@@ -250,25 +270,87 @@ FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const int32_t* s_off,
     const int mt = local / nt, ntile = local - mt * nt;
     T.n0 = ntile * BN;
     const int32_t o0 = s_off[lo], o1 = s_off[lo + 1];
-    if (a.mode == FG8_GROUP_M) {
-        T.rowA = (int64_t)o0 + (int64_t)mt * BM;
-        // rows past M_total (offsets inconsistent with the buffers) are never touched
-        T.rows_valid = (int)max((int64_t)0, min((int64_t)min(BM, (o1 - o0) - mt * BM),
-                                                a.M_total - T.rowA));
-        T.kx0 = 0;
-        T.nkb = a.K / BK;
-        T.rowB = (int64_t)lo * a.N + T.n0;
-        T.out_row0 = T.rowA;
-    } else {
-        T.rowA = (int64_t)mt * BM;
-        T.rows_valid = BM;
-        // contraction range clamped to the operands' width
-        T.kx0 = min(max(o0, 0), a.K) & ~(BK - 1);
-        T.nkb = max(0, min(o1, a.K) - T.kx0) / BK;
-        T.rowB = T.n0;
-        T.out_row0 = (int64_t)lo * a.M_total + T.rowA;
-    }
+    T.rowA = (int64_t)o0 + (int64_t)mt * BM;
+    // rows past M_total (offsets inconsistent with the buffers) are never touched
+    T.rows_valid = (int)max((int64_t)0, min((int64_t)min(BM, (o1 - o0) - mt * BM),
+                                            a.M_total - T.rowA));
+    T.kx0 = 0;
+    T.nkb = a.K / BK;
+    T.rowB = (int64_t)lo * a.N + T.n0;
+    T.out_row0 = T.rowA;
     return T;
+}
+
+// Contraction-grouped: g -> (expert, m-tile, n-tile).  s_order lists the experts
+// in processing order, in groups of `mix` whose tiles alternate; every expert
+// has tpe tiles.
+FG8_DEV Tile decode_tile_k(int g, const int32_t* s_order, const int32_t* s_off, const GemmArgs& a,
+                           int nt, int tpe, int mix) {
+    const int grp = g / (mix * tpe);
+    const int rem = g - grp * mix * tpe;
+    const int e = s_order[grp * mix + rem % mix];
+    const int local = rem / mix;
+    const int mt = local / nt, ntile = local - mt * nt;
+    Tile T;
+    T.e = e;
+    T.n0 = ntile * BN;
+    const int32_t o0 = s_off[e], o1 = s_off[e + 1];
+    T.rowA = (int64_t)mt * BM;
+    T.rows_valid = BM;
+    // contraction range clamped to the operands' width
+    T.kx0 = min(max(o0, 0), a.K) & ~(BK - 1);
+    T.nkb = max(0, min(o1, a.K) - T.kx0) / BK;
+    T.rowB = T.n0;
+    T.out_row0 = (int64_t)e * a.M_total + T.rowA;
+    return T;
+}
+
+// K blocks of expert e in the contraction-grouped mode (as decode_tile_k)
+FG8_DEV int expert_kblocks(const int32_t* s_off, int e, int K) {
+    const int kx0 = min(max(s_off[e], 0), K) & ~(BK - 1);
+    return max(0, min(s_off[e + 1], K) - kx0) / BK;
+}
+
+// tile ring: the producer publishes, the other roles take (bounded waits).
+// An entry is {K blocks, first output row, first output column, 0}; K blocks
+// -1 ends the stream.
+struct TileRing {
+    int4* slots;
+    uint32_t full0, empty0;   // mbarrier addresses of slot 0
+    uint32_t slot = 0, phase = 0;
+    FG8_DEV void advance() {
+        if (++slot == kTileRing) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+FG8_DEV bool ring_wait_free(TileRing& R, volatile int* abort_flag, int32_t* status) {
+    return mbar_wait(R.empty0 + 8u * R.slot, R.phase ^ 1u, abort_flag, status);
+}
+
+FG8_DEV void ring_publish(TileRing& R, int4 v) {
+    asm volatile("st.shared.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(R.slots + R.slot)),
+                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+    mbar_arrive(R.full0 + 8u * R.slot);   // release: the entry is visible to the takers
+    R.advance();
+}
+
+// whole_warp: every lane of the warp calls this (lane 0 releases the slot);
+// otherwise a single thread does.
+FG8_DEV bool ring_take(TileRing& R, bool whole_warp, int4& v, volatile int* abort_flag,
+                       int32_t* status) {
+    if (!mbar_wait(R.full0 + 8u * R.slot, R.phase, abort_flag, status)) return false;
+    asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(R.slots + R.slot))
+                 : "memory");
+    if (whole_warp) __syncwarp();
+    if (!whole_warp || (threadIdx.x & 31) == 0) mbar_arrive(R.empty0 + 8u * R.slot);
+    R.advance();
+    return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -296,6 +378,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+    const uint32_t ring_full0 = bar0 + 8u * (2 * kStages + 5);
+    const uint32_t ring_empty0 = ring_full0 + 8u * kTileRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     int32_t* s_tiles = reinterpret_cast<int32_t*>(smem + kOffTiles);
@@ -315,6 +399,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             mbar_init(tempty_bar(b), kEpiWarps);
         }
         mbar_init(drain_bar, 1);
+        if (kGroupK) {
+            for (int i = 0; i < kTileRing; ++i) {
+                mbar_init(ring_full0 + 8u * i, 1);
+                mbar_init(ring_empty0 + 8u * i, 1 + kEpiWarps);   // MMA thread + promotion warps
+            }
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -326,21 +416,40 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // tiles per expert -> exclusive prefix (in place)
-    for (int e = threadIdx.x; e < a.E; e += kThreads) {
-        const int32_t cnt = a.mode == FG8_GROUP_M
-                                ? (max(0, a.offsets[e + 1] - a.offsets[e]) + BM - 1) / BM
-                                : (int32_t)(a.M_total / BM);
-        s_tiles[e] = cnt * nt;
-    }
     for (int e = threadIdx.x; e <= a.E; e += kThreads) s_off[e] = a.offsets[e];
-    __syncthreads();
-    fg8::block_exclusive_scan(s_tiles, s_tiles, a.E, s_warp);
+    const int mix = (kGroupK && a.E % kMix == 0) ? kMix : 1;
+    const int tpe = (int)(a.M_total / BM) * nt;   // contraction-grouped: tiles per expert
+    if (!kGroupK) {
+        // tiles per expert -> exclusive prefix (in place)
+        for (int e = threadIdx.x; e < a.E; e += kThreads)
+            s_tiles[e] = (max(0, a.offsets[e + 1] - a.offsets[e]) + BM - 1) / BM * nt;
+        __syncthreads();
+        fg8::block_exclusive_scan(s_tiles, s_tiles, a.E, s_warp);
+    } else {
+        // processing order: rank the experts by K blocks (descending, ties by
+        // id); group i takes ranks i, i + E/mix, i + 2E/mix, ... (one per size
+        // quantile)
+        __syncthreads();
+        const int ng = a.E / mix;
+        for (int e = threadIdx.x; e < a.E; e += kThreads) {
+            const int ke = expert_kblocks(s_off, e, a.K);
+            int rank = 0;
+            for (int f = 0; f < a.E; ++f) {
+                const int kf = expert_kblocks(s_off, f, a.K);
+                rank += (kf > ke) || (kf == ke && f < e);
+            }
+            s_tiles[(rank % ng) * mix + rank / ng] = e;
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = s_tiles[a.E];
+    const int total = kGroupK ? a.E * tpe : s_tiles[a.E];
+    TileRing ring;
+    ring.slots = reinterpret_cast<int4*>(smem + L::kOffRing);
+    ring.full0 = ring_full0;
+    ring.empty0 = ring_empty0;
 
     if (warp < kCtrlWarps) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
@@ -350,8 +459,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             uint32_t stage = 0, phase = 0, sc = 0;
             int e_hint = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
+            for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
+                Tile T;
+                if (kGroupK) {
+                    if (!ring_wait_free(ring, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tile = (int)atomicAdd(a.tile_ctr, 1u);
+                    if (tile >= total || tile < 0) {
+                        ring_publish(ring, make_int4(-1, 0, 0, 0));
+                        break;
+                    }
+                    T = decode_tile_k(tile, s_tiles, s_off, a, nt, tpe, mix);
+                    ring_publish(ring, make_int4(T.nkb, (int)T.out_row0, T.n0, 0));
+                } else {
+                    if ((tile += gridDim.x) >= total) break;
+                    T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
+                }
                 for (int kb = 0; kb < T.nkb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.status)) {
                         ok = false;
@@ -376,6 +501,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         phase ^= 1u;
                     }
                 }
+                if (!ok) break;
             }
             if (!ok) {
                 // let copies already issued land before the CTA winds down
@@ -393,9 +519,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
             int e_hint = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
-                for (int kb = 0; kb < T.nkb; ++kb) {
+            for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
+                int nkb;
+                if (kGroupK) {
+                    int4 v;
+                    if (!ring_take(ring, false, v, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (v.x < 0) break;
+                    nkb = v.x;
+                } else {
+                    if ((tile += gridDim.x) >= total) break;
+                    nkb = decode_tile(tile, s_tiles, s_off, a, nt, e_hint).nkb;
+                }
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(tempty_bar(buf), bphase ^ 1u, abort_flag, a.status) ||
                         !mbar_wait(full_bar(stage), phase, abort_flag, a.status)) {
                         ok = false;
@@ -417,6 +555,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     buf ^= 1u;
                     if (buf == 0) bphase ^= 1u;
                 }
+                if (!ok) break;
             }
             // all MMAs issued by this thread are complete once drain_bar flips
             mma_commit(drain_bar);
@@ -438,21 +577,42 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t nbox = 0;    // TMA-store boxes issued by this warp (contraction-grouped)
         int e_hint = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
+            int4 v = make_int4(0, 0, 0, 0);
+            if (kGroupK) {
+                if (!ring_take(ring, true, v, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                if (v.x < 0) break;
+            } else if ((tile += gridDim.x) >= total) {
+                break;
+            }
             float2 acc[64];   // columns 2i, 2i + 1 of this thread's 128-column half
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            // Only what the K loop needs stays live through it; the epilogue
-            // decodes the tile again (registers are the promotion's limit).
-            int nkb;
+            // Only what the K loop and the epilogue need stays live (registers
+            // are the promotion's limit); output rows fit in 32 bits (checked
+            // on the host).
+            int nkb, rows_valid, out_row0, col0;
             bool row_ok, col_ok;
             const float* sa_p;
             const float* sb_p;
-            {
+            if (kGroupK) {
+                nkb = v.x;
+                rows_valid = BM;
+                out_row0 = v.y;
+                row_ok = true;
+                col0 = v.z + 128 * half;
+                col_ok = col0 < a.N;
+                sa_p = sb_p = nullptr;
+            } else {
                 const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
                 nkb = T.nkb;
+                rows_valid = T.rows_valid;
+                out_row0 = (int)T.out_row0;
                 row_ok = r < T.rows_valid;
-                const int col0 = T.n0 + 128 * half;
+                col0 = T.n0 + 128 * half;
                 col_ok = col0 < a.N;
                 sa_p = a.sa + T.rowA + r;
                 sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
@@ -540,40 +700,43 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (buf == 0) bphase ^= 1u;
             }
             if (!ok) break;
-            const Tile T = decode_tile(tile, s_tiles, s_off, a, nt, e_hint);
-            const int col0 = T.n0 + 128 * half;
             if (kGroupK) {
                 // Epilogue (contraction-grouped, fp32, full 128-row tiles): each
-                // warp writes its 32 rows x 128 columns as four 32 x 32 boxes
-                // through two 4 KB staging buffers and TMA-stores them; the stores
-                // drain while the warp moves on to the next tile's promotion.
+                // warp writes its 32 rows x 128 columns as four 32 x 32 boxes,
+                // two at a time through its two 4 KB staging buffers, and
+                // TMA-stores them; the stores drain while the warp moves on.
                 // 128-byte swizzle: 16-byte chunk c of box row rr sits at chunk
                 // c ^ (rr & 7); the four lanes of a row write 32 contiguous bytes,
                 // so each 8-byte store of the warp is two conflict-free wavefronts.
                 if (col_ok) {
 #pragma unroll
-                    for (int bx = 0; bx < 4; ++bx) {
-                        const uint32_t b = (uint32_t)(nbox & 1);
-                        if (lane == 0 && nbox >= 2) bulk_wait_read<1>();   // buffer b drained
+                    for (int pr = 0; pr < 2; ++pr) {
+                        if (lane == 0 && nbox > 0) bulk_wait_read<0>();   // both buffers drained
                         __syncwarp();
-                        uint8_t* box = smem + kOffStage + ep * kTmaStagePerWarp + b * kBoxBytes;
-                        const int cg = bx >> 1;
+                        uint8_t* stg = smem + kOffStage + ep * kTmaStagePerWarp;
 #pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            const int j = 4 * (bx & 1) + jj;
-                            const int chunk = 2 * jj + ((lane & 3) >> 1);
+                        for (int bb = 0; bb < 2; ++bb) {
+                            const int bx = 2 * pr + bb;   // box: columns 32 bx .. of the half
+                            uint8_t* box = stg + bb * kBoxBytes;
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const int rr = g4 + 8 * k;
-                                *reinterpret_cast<float2*>(box + rr * 128 + ((chunk ^ (rr & 7)) << 4) +
-                                                           8 * (lane & 1)) = acc[(cg * 8 + j) * 4 + k];
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const int j = 4 * (bx & 1) + jj;
+                                const int chunk = 2 * jj + ((lane & 3) >> 1);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int rr = g4 + 8 * k;
+                                    *reinterpret_cast<float2*>(box + rr * 128 + ((chunk ^ (rr & 7)) << 4) +
+                                                               8 * (lane & 1)) = acc[(pr * 8 + j) * 4 + k];
+                                }
                             }
                         }
                         fence_async_shared();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_2d(&tmOut, smem_u32(box), col0 + 32 * bx,
-                                         (int)(T.out_row0 + 32 * quarter));
+#pragma unroll
+                            for (int bb = 0; bb < 2; ++bb)
+                                tma_store_2d(&tmOut, smem_u32(stg + bb * kBoxBytes), col0 + 64 * pr + 32 * bb,
+                                             out_row0 + 32 * quarter);
                             bulk_commit();
                         }
                         ++nbox;
@@ -602,8 +765,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         for (int g = 0; g < 4; ++g) {
                             const int rr = 8 * g + sub;
                             const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
-                            if (32 * quarter + rr < T.rows_valid)
-                                *reinterpret_cast<uint4*>(ob + (T.out_row0 + 32 * quarter + rr) * a.N + 16 * ch) = v;
+                            if (32 * quarter + rr < rows_valid)
+                                *reinterpret_cast<uint4*>(ob + (int64_t)(out_row0 + 32 * quarter + rr) * a.N + 16 * ch) = v;
                         }
                         __syncwarp();
                     }
@@ -622,8 +785,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         for (int g = 0; g < 4; ++g) {
                             const int rr = 8 * g + sub;
                             const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
-                            if (32 * quarter + rr < T.rows_valid)
-                                *reinterpret_cast<uint4*>(ob + (T.out_row0 + 32 * quarter + rr) * a.N + 32 * ch) = v;
+                            if (32 * quarter + rr < rows_valid)
+                                *reinterpret_cast<uint4*>(ob + (int64_t)(out_row0 + 32 * quarter + rr) * a.N + 32 * ch) = v;
                         }
                         __syncwarp();
                     }
@@ -652,6 +815,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     return fg8h::make_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, 128,
                                     box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// contraction-grouped tile counters (one per launch in flight, see kCtrSlots)
+__device__ unsigned int g_tile_ctr[kCtrSlots];
+std::atomic<void*> g_tile_ctr_addr[64];
+std::atomic<unsigned> g_tile_ctr_next{0};
+
+// A zeroed counter for one launch on `stream`, or nullptr on a CUDA error.
+unsigned int* take_tile_counter(cudaStream_t stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    void* base = (dev >= 0 && dev < 64) ? g_tile_ctr_addr[dev].load() : nullptr;
+    if (base == nullptr) {
+        if (cudaGetSymbolAddress(&base, g_tile_ctr) != cudaSuccess) return nullptr;
+        if (dev >= 0 && dev < 64) g_tile_ctr_addr[dev].store(base);
+    }
+    unsigned int* ctr = static_cast<unsigned int*>(base) + g_tile_ctr_next.fetch_add(1) % kCtrSlots;
+    if (cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream) != cudaSuccess) return nullptr;
+    return ctr;
 }
 
 }  // namespace
@@ -724,6 +906,11 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     args.out_f32 = out_dtype == FG8_OUT_F32;
     args.out = out;
     args.status = dev_status;
+    args.tile_ctr = nullptr;
+    if (group_mode == FG8_GROUP_K) {
+        args.tile_ctr = take_tile_counter((cudaStream_t)stream);
+        if (args.tile_ctr == nullptr) return FG8_ERR_CUDA;
+    }
     int64_t grid = fg8h::num_sms();
     if (grid > max_tiles) grid = max_tiles;
     if (grid < 1) grid = 1;

@@ -197,6 +197,10 @@ fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N
  *            sa and sb 16-byte aligned (the scale vectors are bulk-copied);
  *            out_dtype must be FG8_OUT_F32 (weight gradients are accumulated
  *            in fp32; other dtypes return FG8_ERR_UNSUPPORTED).
+ *   The tiles are handed out at run time from a tile counter that the
+ *   library keeps in device memory (64 per device, used in turn and zeroed
+ *   on `stream` before each launch): at most 64 contraction-grouped launches
+ *   may execute at the same time on one device.
  *
  * The fp32 output is the accumulator; the bf16 output is its round-to-
  * nearest-even conversion.  dev_status may be NULL only if no device-side
