@@ -246,10 +246,10 @@ class Step:
             self.status, sp)))
 
         def wquant():
-            fg8.fg8_quantize_weight(u16(self.w_up), E, N, K, self.wq_up, self.sw_up, sp)
+            fg8.fg8_quantize_weight(u16(self.w_up), E, N, K, self.wq_up, self.sw_up, self.status, sp)
             n[0] += 1
             if I:
-                fg8.fg8_quantize_weight(u16(self.w_down), E, K, I, self.wq_dn, self.sw_dn, sp)
+                fg8.fg8_quantize_weight(u16(self.w_down), E, K, I, self.wq_dn, self.sw_dn, self.status, sp)
                 n[0] += 1
         timed("quant_weight", wquant)
         timed("gemm_fprop_up", launch(lambda: fg8.fg8_grouped_gemm(

@@ -72,7 +72,7 @@ def lib() -> ctypes.CDLL:
         L.fg8_colwise_capacity.restype = _I64
         L.fg8_colwise_capacity.argtypes = [_I64, _I]
         L.fg8_quantize_weight.restype = _I
-        L.fg8_quantize_weight.argtypes = [_P, _I, _I, _I, _P, _P, _P]
+        L.fg8_quantize_weight.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P]
         L.fg8_transpose_blockq.restype = _I
         L.fg8_transpose_blockq.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P]
         L.fg8_grouped_gemm.restype = _I
@@ -149,8 +149,9 @@ def fg8_colwise_capacity(R: int, E: int) -> int:
     return lib().fg8_colwise_capacity(R, E)
 
 
-def fg8_quantize_weight(w, E, N, K, wq, sw, stream=None):
-    _check(lib().fg8_quantize_weight(_ptr(w), E, N, K, _ptr(wq), _ptr(sw), _stream(stream)),
+def fg8_quantize_weight(w, E, N, K, wq, sw, dev_status=None, stream=None):
+    _check(lib().fg8_quantize_weight(_ptr(w), E, N, K, _ptr(wq), _ptr(sw), _ptr(dev_status),
+                                     _stream(stream)),
            "fg8_quantize_weight")
 
 
@@ -243,12 +244,12 @@ def quantize_act_colwise(x: torch.Tensor, offsets: torch.Tensor, k: int = 1,
     return xqT, saT, padoff
 
 
-def quantize_weight(w: torch.Tensor, stream=None):
+def quantize_weight(w: torch.Tensor, status=None, stream=None):
     """128x128 block quantize of bf16 w [E,N,K] -> (wq, sw [E,N/128,K/128])."""
     E, N, K = w.shape
     wq = torch.empty((E, N, K), dtype=torch.uint8, device=w.device)
     sw = torch.empty((E, N // 128, K // 128), dtype=torch.float32, device=w.device)
-    fg8_quantize_weight(_u16(w), E, N, K, wq, sw, stream)
+    fg8_quantize_weight(_u16(w), E, N, K, wq, sw, status, stream)
     return wq, sw
 
 

@@ -149,12 +149,16 @@ int64_t fg8_colwise_capacity(int64_t R, int E);
 /*
  * fg8_quantize_weight -- 128x128 block quantization of the weights of all
  * experts in one launch ([K2] FP8 paragraph; [DS] sec. 2.2 128x128 blocks).
- *   w   bf16 [E][N][K], N % 128 == 0, K % 128 == 0
- *   wq  E4M3 [E][N][K]
+ *   w   bf16 [E][N][K], N % 128 == 0, K % 128 == 0, 16-byte aligned
+ *   wq  E4M3 [E][N][K], 16-byte aligned
  *   sw  fp32 [E][N/128][K/128]
+ *   dev_status  optional (NULL allowed) device int32: a block whose load
+ *       never arrives (bounded wait) gets a NaN scale and FG8_ERR_TIMEOUT
+ *       is recorded here.
  */
 fg8_status fg8_quantize_weight(const uint16_t* w, int E, int N, int K,
-                               uint8_t* wq, float* sw, fg8_stream_t stream);
+                               uint8_t* wq, float* sw, int32_t* dev_status,
+                               fg8_stream_t stream);
 
 /*
  * fg8_transpose_blockq -- transpose an already block-quantized weight and its

@@ -50,9 +50,9 @@ def test_sizes(L):
 def test_null_and_shape_arguments_rejected_on_host(L):
     INV = fg8.FG8_ERR_INVALID_ARG
     # null pointers / bad sizes return before any CUDA call
-    assert L.fg8_quantize_weight(None, 1, 128, 128, None, None, None) == INV
-    assert L.fg8_quantize_weight(16, 1, 100, 128, 16, 16, None) == INV        # N % 128
-    assert L.fg8_quantize_weight(16, 0, 128, 128, 16, 16, None) == INV        # E < 1
+    assert L.fg8_quantize_weight(None, 1, 128, 128, None, None, None, None) == INV
+    assert L.fg8_quantize_weight(16, 1, 100, 128, 16, 16, None, None) == INV        # N % 128
+    assert L.fg8_quantize_weight(16, 0, 128, 128, 16, 16, None, None) == INV        # E < 1
     assert L.fg8_transpose_blockq(None, None, 1, 128, 128, None, None, None) == INV
     assert L.fg8_transpose_blockq(16, 16, 1, 128, 130, 16, 16, None) == INV  # K % 128
     assert L.fg8_grouped_gemm(None, None, None, None, None, 128, 128, 128, 1, 0, 0, 0, None,
@@ -64,7 +64,7 @@ def test_null_and_shape_arguments_rejected_on_host(L):
     assert L.fg8_quantize_act(16, 10, 100, None, 1, 1, None, 1, 16, 16, None, None, None,
                               None, None, None, 0, None, None) == INV         # K % 128
     # misaligned FP8 / bf16 buffers
-    assert L.fg8_quantize_weight(18, 1, 128, 128, 16, 16, None) == INV
+    assert L.fg8_quantize_weight(18, 1, 128, 128, 16, 16, None, None) == INV
     assert L.fg8_grouped_gemm(17, 16, 16, 16, 16, 128, 128, 128, 1, 0, 0, 0, 16, None,
                               None) == INV
     # unsupported combinations
