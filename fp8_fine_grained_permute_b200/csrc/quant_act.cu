@@ -14,17 +14,23 @@
 //         maps, then quantizes each of its token rows ONCE and stores the
 //         codes to all k destination rows.
 //    Phases are separated by grid-wide barriers with bounded waits.
-//  * quant_rows    (rows already in expert order): the phase-C row loop only.
-//  * colwise_tiles (weight-gradient operands): 128 tokens x 128 columns per
-//    CTA, amax per column over the tile's tokens, codes written transposed so
-//    that the token axis is contiguous (thread = 2 columns x 32 tokens).
+//  * quant_rows    (rows already in expert order): 128 x 128 boxes staged in
+//    shared memory by one TMA load each, a half-warp per row tile.
+//  * colwise_tiles (weight-gradient operands): one 128-token tile x a quarter
+//    of the columns per CTA, 128 columns at a time through a two-stage
+//    cp.async pipeline; amax per column over the tile's tokens, codes written
+//    transposed so that the token axis is contiguous (thread = 2 columns x 32
+//    tokens).
+#include <cuda.h>
+
 #include <atomic>
 
 #include "fg8_common.cuh"
+#include "fg8_tma.cuh"
 
 namespace {
 
-constexpr int kThreads = 512;            // route_quant / quant_rows
+constexpr int kThreads = 512;            // route_quant
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 2048;               // experts supported by route_quant / colwise
 constexpr int kMaxGrid = 1024;            // CTAs of route_quant (sizes the workspace)
@@ -199,14 +205,49 @@ __global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
 // identity mode
 // --------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(kThreads, 2)
-quant_rows(const uint16_t* __restrict__ x, int64_t R, int64_t K, uint8_t* __restrict__ xq,
-           float* __restrict__ sa) {
-    const int lane = threadIdx.x & 31;
-    const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
-    for (int64_t r = gw; r < R; r += nwarps)
-        quant_row(x + r * K, K, lane == 0 ? (int)r : -1, 1, xq, sa, R, lane);
+// One CTA per 128 rows x 128 columns: one 2-D TMA load stages the box (32 KB,
+// rows past R read as zeros) in shared memory, five CTAs per SM keep the
+// loads in flight.  A half-warp owns one row's 1x128 tile at a time (16 lanes
+// x 8 values): amax by a 4-step shuffle, then the bracketed fast path.
+constexpr int kRowThreads = 256;
+constexpr uint32_t kRowBoxBytes = 128 * 256;
+
+__global__ void __launch_bounds__(kRowThreads, 5)
+quant_rows(const __grid_constant__ CUtensorMap tmX, int64_t R, int64_t K, uint8_t* __restrict__ xq,
+           float* __restrict__ sa, int32_t* status) {
+    extern __shared__ __align__(128) uint8_t box[];   // [128 rows][256 bytes]
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_abort;
+    const int kb = blockIdx.x;
+    const int64_t r0 = (int64_t)blockIdx.y * 128;
+    const int t = threadIdx.x;
+    const uint32_t bar = fg8::tma::smem_u32(&s_bar);
+    if (t == 0) {
+        s_abort = 0;
+        fg8::tma::mbar_init(bar, 1);
+        fg8::tma::fence_barrier_init();
+        fg8::tma::mbar_arrive_expect_tx(bar, kRowBoxBytes);
+        fg8::tma::tma_load_2d(&tmX, fg8::tma::smem_u32(box), bar, kb * 128, (int)r0);
+    }
+    __syncthreads();
+    if (!fg8::tma::mbar_wait(bar, 0, &s_abort, status)) return;   // block-uniform in practice
+    const int half = t >> 4;       // 16 half-warps: rows half + 16 i
+    const int l = t & 15;          // 16-byte piece of the row's tile
+#pragma unroll 2
+    for (int i = 0; i < 8; ++i) {
+        const int rr = half + 16 * i;
+        const uint4 v = *reinterpret_cast<const uint4*>(box + rr * 256 + l * 16);
+        float m = fg8::amax8(v);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+        const float sc = fg8::tile_scale(m);
+        const uint2 c = fg8::quant8(v, fg8::make_qscale(sc));
+        const int64_t r = r0 + rr;
+        if (r < R) {
+            *reinterpret_cast<uint2*>(xq + r * K + (int64_t)kb * 128 + l * 8) = c;
+            if (l == 0) sa[(int64_t)kb * R + r] = sc;
+        }
+    }
 }
 
 // --------------------------------------------------------------------------
@@ -227,20 +268,38 @@ struct ColArgs {
     uint8_t* xqT;
     float* saT;
     int32_t* padoff_out;
+    int32_t* status;
 };
 
-// One CTA per (128-token tile of one expert) x (128 columns).  Thread t owns
-// the column pair p = t % 64 (columns 2p, 2p+1) for the 32 tokens of quarter
-// q = t / 64: it loads them as 32-bit words (a warp load is one 128-byte row
-// piece), reduces its two column maxima in registers (16-bit SIMD max), and
-// the four quarters of a pair combine through shared memory.  Codes are then
-// formed per column on 8 consecutive tokens at a time (bracketed fast path)
-// and stored transposed: 32 contiguous bytes of each column per thread.
-__global__ void __launch_bounds__(kColThreads) colwise_tiles(ColArgs a) {
+// One CTA per 128-token tile of one expert and per group of 128-column blocks
+// (a quarter of the columns).  The tile's source rows (contiguous, or gathered
+// through row_map) are found once; then, for each column block in turn, the
+// 128 x 256-byte slice is brought into shared memory by cp.async (16 bytes a
+// thread-copy, padding rows zero-filled), two stages deep, so the next block's
+// data is in flight while this one is converted.  Thread t owns the column
+// pair p = t % 64 (columns 2p, 2p+1) for the 32 tokens of quarter q = t / 64:
+// it reads them as 32-bit words (a warp reads one 128-byte row piece,
+// conflict-free), reduces its two column maxima in registers (16-bit SIMD
+// max), and the four quarters of a pair combine through shared memory.  Codes
+// are then formed per column on 8 consecutive tokens at a time (bracketed
+// fast path) and stored transposed: 32 contiguous bytes (a whole sector) of
+// each column per thread.  (Measured against one CTA per 128 x 128 tile, with
+// the expert prefix recomputed by every CTA: 25% slower.)
+constexpr uint32_t kColTileBytes = 128 * 256;
+constexpr int kColCtasPerSm = 3;
+constexpr int kColGroups = 4;      // column groups per tile (grid.y)
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColArgs a) {
+    extern __shared__ __align__(128) uint8_t s_tile[];   // [2][128 rows][256 bytes]
     __shared__ int32_t s_pref[kMaxE + 1];
     __shared__ int32_t s_warp[33];
     __shared__ int32_t s_rows[128];
-    __shared__ uint32_t s_amax[4][64];
+    __shared__ uint32_t s_amax[2][4][64];
 
     const int t = threadIdx.x;
     const int E = a.E;
@@ -255,21 +314,18 @@ __global__ void __launch_bounds__(kColThreads) colwise_tiles(ColArgs a) {
 
     const int tile = blockIdx.x;
     if (tile >= s_pref[E]) return;   // block-uniform
-    int lo = 0, hi = E;              // largest e with s_pref[e] <= tile
+    int lo = 0, hi = E;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (s_pref[mid] <= tile) lo = mid; else hi = mid;
     }
     const int e = lo;
     const int tb = tile - s_pref[e];
-    const int64_t pcol = (int64_t)128 * s_pref[e] + 128 * tb;   // padded token column
-    if (pcol + 128 > a.P) return;   // offsets inconsistent with R: never write past the buffers
+    const int64_t pcol = (int64_t)128 * s_pref[e] + 128 * tb;
+    if (pcol + 128 > a.P) return;
     const int32_t Te = a.offsets[e + 1] - a.offsets[e];
     const int n_in = min(128, Te - 128 * tb);
     const int64_t row0 = (int64_t)a.offsets[e] + 128 * tb;
-    const int64_t col0 = (int64_t)blockIdx.y * 128;
-
-    // source rows of the tile's 128 tokens (-1: padding or out of range)
     if (t < 128) {
         const int64_t lr = row0 + t;
         int32_t sr = -1;
@@ -280,46 +336,73 @@ __global__ void __launch_bounds__(kColThreads) colwise_tiles(ColArgs a) {
         s_rows[t] = sr;
     }
     __syncthreads();
-
+    // this CTA's column blocks
+    const int ncb = (int)(a.C / 128);
+    const int cb0 = (int)((int64_t)ncb * blockIdx.y / gridDim.y), cb1 = (int)((int64_t)ncb * (blockIdx.y + 1) / gridDim.y);
+    // per thread: its 8 pieces' source rows are fixed for the tile
+    const uint16_t* srcp[8];
+    uint32_t nbytes[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int u = t + kColThreads * j;
+        const int32_t sr = s_rows[u >> 4];
+        srcp[j] = a.x + (sr >= 0 ? (int64_t)sr * a.C + (u & 15) * 8 : 0);
+        nbytes[j] = sr >= 0 ? 16u : 0u;
+    }
+    auto issue = [&](int cb, int st) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int u = t + kColThreads * j;
+            cp_async16(fg8::tma::smem_u32(s_tile + st * kColTileBytes + (u >> 4) * 256 + (u & 15) * 16),
+                       srcp[j] + (nbytes[j] ? (int64_t)cb * 128 : 0), nbytes[j]);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
     const int p = t & 63, q = t >> 6;
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(a.x + col0) + p;
-    const int64_t wstride = a.C / 2;    // 32-bit words per source row
-    uint32_t w[32];
+    if (cb0 < cb1) issue(cb0, 0);
+    for (int cb = cb0; cb < cb1; ++cb) {
+        const int st = (cb - cb0) & 1;
+        if (cb + 1 < cb1) {
+            issue(cb + 1, st ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        const int64_t col0 = (int64_t)cb * 128;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(s_tile + st * kColTileBytes) + p;
+        uint32_t w[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int32_t sr = s_rows[32 * q + i];
-        w[i] = sr >= 0 ? __ldg(src + (int64_t)sr * wstride) : 0u;
+        for (int i = 0; i < 32; ++i) w[i] = src[(32 * q + i) * 64];
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+        s_amax[st][q][p] = m;
+        __syncthreads();   // amax of this stage complete; also: every thread is done reading the other stage
+        m = __vmaxu2(__vmaxu2(s_amax[st][0][p], s_amax[st][1][p]), __vmaxu2(s_amax[st][2][p], s_amax[st][3][p]));
+        const float s0 = fg8::tile_scale(__uint_as_float((m & 0xFFFFu) << 16));
+        const float s1 = fg8::tile_scale(__uint_as_float(m & 0xFFFF0000u));
+        const fg8::QScale q0 = fg8::make_qscale(s0), q1 = fg8::make_qscale(s1);
+        uint4 v0[4], v1[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            v0[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x5410), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x5410),
+                               __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x5410), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x5410));
+            v1[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x7632), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x7632),
+                               __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x7632), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x7632));
+        }
+        uint2 c0[4], c1[4];
+        fg8::quant8xN<4>(v0, q0, c0);
+        fg8::quant8xN<4>(v1, q1, c1);
+        uint8_t* d0 = a.xqT + (col0 + 2 * p) * a.P + pcol + 32 * q;
+        uint8_t* d1 = d0 + a.P;
+        reinterpret_cast<uint4*>(d0)[0] = make_uint4(c0[0].x, c0[0].y, c0[1].x, c0[1].y);
+        reinterpret_cast<uint4*>(d0)[1] = make_uint4(c0[2].x, c0[2].y, c0[3].x, c0[3].y);
+        reinterpret_cast<uint4*>(d1)[0] = make_uint4(c1[0].x, c1[0].y, c1[1].x, c1[1].y);
+        reinterpret_cast<uint4*>(d1)[1] = make_uint4(c1[2].x, c1[2].y, c1[3].x, c1[3].y);
+        if (q == 0)
+            reinterpret_cast<float2*>(a.saT + (pcol / 128) * a.C + col0)[p] = make_float2(s0, s1);
     }
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-    s_amax[q][p] = m;
-    __syncthreads();
-    m = __vmaxu2(__vmaxu2(s_amax[0][p], s_amax[1][p]), __vmaxu2(s_amax[2][p], s_amax[3][p]));
-    const float s0 = fg8::tile_scale(__uint_as_float((m & 0xFFFFu) << 16));   // column 2p
-    const float s1 = fg8::tile_scale(__uint_as_float(m & 0xFFFF0000u));       // column 2p + 1
-    const fg8::QScale q0 = fg8::make_qscale(s0), q1 = fg8::make_qscale(s1);
-
-    // per column: 4 groups of 8 consecutive tokens, bf16 pairs regrouped by column
-    uint4 v0[4], v1[4];
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        v0[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x5410), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x5410),
-                           __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x5410), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x5410));
-        v1[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x7632), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x7632),
-                           __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x7632), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x7632));
-    }
-    uint2 c0[4], c1[4];
-    fg8::quant8xN<4>(v0, q0, c0);
-    fg8::quant8xN<4>(v1, q1, c1);
-    uint8_t* d0 = a.xqT + (col0 + 2 * p) * a.P + pcol + 32 * q;
-    uint8_t* d1 = d0 + a.P;
-    reinterpret_cast<uint4*>(d0)[0] = make_uint4(c0[0].x, c0[0].y, c0[1].x, c0[1].y);
-    reinterpret_cast<uint4*>(d0)[1] = make_uint4(c0[2].x, c0[2].y, c0[3].x, c0[3].y);
-    reinterpret_cast<uint4*>(d1)[0] = make_uint4(c1[0].x, c1[0].y, c1[1].x, c1[1].y);
-    reinterpret_cast<uint4*>(d1)[1] = make_uint4(c1[2].x, c1[2].y, c1[3].x, c1[3].y);
-    if (q == 0)
-        reinterpret_cast<float2*>(a.saT + (pcol / 128) * a.C + col0)[p] = make_float2(s0, s1);
 }
 
 size_t ws_layout(int64_t E, size_t* off_totals, size_t* off_chunks) {
@@ -370,11 +453,17 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
         if (T == 0) return FG8_OK;
         if (!xq || !sa) return FG8_ERR_INVALID_ARG;
         if (!fg8h::aligned16(xq) || (reinterpret_cast<uintptr_t>(sa) & 3)) return FG8_ERR_INVALID_ARG;
-        const int64_t warps_needed = T;
-        int64_t blocks = (warps_needed + kWarps - 1) / kWarps;
-        const int64_t cap = (int64_t)fg8h::num_sms() * 4;
-        if (blocks > cap) blocks = cap;
-        quant_rows<<<(unsigned)blocks, kThreads, 0, st>>>(x, T, K, xq, sa);
+        if (K / 128 > INT32_MAX || (T + 127) / 128 > 65535 || T > INT32_MAX)
+            return FG8_ERR_UNSUPPORTED;
+        CUtensorMap m;
+        if (!fg8h::make_tensor_map_2d(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, (uint64_t)T,
+                                      (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return FG8_ERR_CUDA;
+        if (cudaFuncSetAttribute(quant_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kRowBoxBytes) != cudaSuccess)
+            return FG8_ERR_CUDA;
+        dim3 grid((unsigned)(K / 128), (unsigned)((T + 127) / 128));
+        quant_rows<<<grid, kRowThreads, kRowBoxBytes, st>>>(m, T, K, xq, sa, dev_status);
         return fg8h::launch_status();
     }
 
@@ -425,9 +514,12 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
         if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
         ColArgs a;
         a.x = x; a.T_src = T; a.R = R; a.C = K; a.row_map = row_token; a.offsets = offsets_in; a.E = E; a.P = P;
-        a.xqT = xqT; a.saT = saT; a.padoff_out = offsets_out;
-        dim3 grid((unsigned)max_tiles, (unsigned)(K / 128));
-        colwise_tiles<<<grid, kColThreads, 0, st>>>(a);
+        a.xqT = xqT; a.saT = saT; a.padoff_out = offsets_out; a.status = dev_status;
+        if (cudaFuncSetAttribute(colwise_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(2 * kColTileBytes)) != cudaSuccess)
+            return FG8_ERR_CUDA;
+        dim3 grid((unsigned)max_tiles, (unsigned)kColGroups);
+        colwise_tiles<<<grid, kColThreads, 2 * kColTileBytes, st>>>(a);
         return fg8h::launch_status();
     }
     return FG8_ERR_INVALID_ARG;
