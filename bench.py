@@ -126,18 +126,18 @@ def work_of(cfg: W.MoEConfig, padded_total: int):
 TRAFFIC_CAPTURE = {
     "config": "kanana",
     "families": {
-        "quant_act_permute": (228.7e6, "quant_act", "afcb9e785c95"),
-        "quant_weight": (792.6e6, "quant_weight", "5af2cf679f5d"),
-        "gemm_fprop_up": (680.7e6, "gemm", "9ea80bdb42f9"),
-        "gemm_fprop_down": (530.0e6, "gemm", "9ea80bdb42f9"),
-        "transpose_blockq": (348.3e6, "transpose", "c1e4961cfa8c"),
-        "quant_act_rows": (593.2e6, "quant_act", "afcb9e785c95"),
-        "gemm_dgrad": (722.6e6, "gemm", "9ea80bdb42f9"),
-        "quant_act_colwise": (662.3e6, "quant_act", "afcb9e785c95"),
-        "gemm_wgrad": (1152.2e6, "gemm", "9ea80bdb42f9"),
+        "quant_act_permute": (224.8e6, "quant_act", "20970841eab1"),
+        "quant_weight": (840.1e6, "quant_weight", "0c431cbcafdb"),
+        "gemm_fprop_up": (679.4e6, "gemm", "5b9d1343ec4e"),
+        "gemm_fprop_down": (529.6e6, "gemm", "5b9d1343ec4e"),
+        "transpose_blockq": (345.9e6, "transpose", "c1e4961cfa8c"),
+        "quant_act_rows": (624.2e6, "quant_act", "20970841eab1"),
+        "gemm_dgrad": (721.7e6, "gemm", "5b9d1343ec4e"),
+        "quant_act_colwise": (663.4e6, "quant_act", "20970841eab1"),
+        "gemm_wgrad": (1150.7e6, "gemm", "5b9d1343ec4e"),
     },
 }
-_SRC = {"quant_act": ["quant_act.cu"], "quant_weight": ["quant_weight.cu"],
+_SRC = {"quant_act": ["quant_act.cu", "fg8_tma.cuh"], "quant_weight": ["quant_weight.cu", "fg8_tma.cuh"],
         "transpose": ["transpose_blockq.cu"], "gemm": ["grouped_gemm.cu", "fg8_tma.cuh"]}
 
 
