@@ -49,24 +49,35 @@ namespace {
 
 using namespace fg8::tma;
 
+// 128 x 256 tiles: N = 256 is the widest single-CTA tcgen05.mma, and narrower
+// ones do not pay (128 x 128 tiles with four TMEM buffers were measured at
+// 0.6x the throughput: an N = 128 MMA takes nearly as long as an N = 256 one).
 constexpr int BM = 128, BN = 256, BK = 128;
 constexpr uint32_t kABytes = BM * BK;              // 16 KB
 constexpr uint32_t kBBytes = BN * BK;              // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kEpiWarps = 8;                       // two promotion warpgroups
 constexpr int kCtrlWarps = 4;                      // warpgroup 0: TMA, MMA, 2 idle warps
-constexpr int kThreads = 32 * (kCtrlWarps + kEpiWarps);   // 384
+// Promotion warps: two warpgroups of 128 columns each, in both modes.  (Four
+// warpgroups of 64 columns, at 112 registers, were measured slower for the
+// row-grouped mode: 2.85 -> 3.94 ms on the DeepSeek-shaped fprop, so the packed
+// FMA work, not latency, bounds the promotion there.)
 // Register split (setmaxnreg): the control warpgroup gives registers back and
-// the promotion warpgroups take them, so each promotion thread can hold its
-// 128 accumulators and 64 partial sums in flight.  The split must not exceed
-// what the CTA was launched with (threads x registers per thread), or the
-// increase would wait forever: 128 x 40 + 256 x 232 = 64512 = 384 x 168.  The
-// host refuses to launch unless the compiled kernel has >= kLaunchRegs.
-constexpr int kCtrlRegs = 40;
-constexpr int kEpiRegs = 232;
-constexpr int kLaunchRegs = 168;
-static_assert(32 * kCtrlWarps * kCtrlRegs + 32 * kEpiWarps * kEpiRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
+// the promotion warpgroups take them.  The split must not exceed what the CTA
+// was launched with (threads x registers per thread), or the increase would
+// wait forever; the host refuses to launch unless the compiled kernel has
+// >= kLaunchRegs.
+template <bool kGroupK>
+struct Warps {
+    static constexpr int kEpiWarps = 8;
+    static constexpr int kThreads = 32 * (kCtrlWarps + kEpiWarps);   // 384
+    static constexpr int kCols = BN / (kEpiWarps / 4);               // columns per promotion warp
+    static constexpr int kCtrlRegs = 40;
+    static constexpr int kEpiRegs = 232;
+    static constexpr int kLaunchRegs = 168;
+    static_assert(32 * kCtrlWarps * kCtrlRegs + 32 * kEpiWarps * kEpiRegs <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+    static_assert(kLaunchRegs * kThreads <= 65536, "launch allocation exceeds the register file");
+};
 constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;                // two partial buffers of BN columns
 
@@ -124,7 +135,7 @@ struct Layout {
     static constexpr uint32_t kOffWarp = kOffOffs + 4 * (kMaxE + 4);    // int32 [36]
     static constexpr uint32_t kOffStage = align_up(kOffWarp + 4 * 36, kGroupK ? 1024 : 16);
     static constexpr uint32_t kStageAll =
-        kEpiWarps * (kGroupK ? kTmaStagePerWarp : kStagePerWarp);
+        Warps<kGroupK>::kEpiWarps * (kGroupK ? kTmaStagePerWarp : kStagePerWarp);
     static constexpr uint32_t kOffScales = kOffStage + kStageAll;
     static constexpr uint32_t kSmemBytes =
         kOffScales + (kGroupK ? kScaleSlots * kScaleSlotBytes : 0) + 1024;   // + alignment slack
@@ -186,23 +197,9 @@ FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;"
 // tcgen05.wait::ld, so no use can be scheduled before the wait).
 FG8_DEV void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n"
         "tcgen05.wait::ld.sync.aligned;\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
-          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
-          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
-          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
-          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
-          "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
 }
@@ -358,11 +355,13 @@ FG8_DEV bool ring_take(TileRing& R, bool whole_warp, int4& v, volatile int* abor
 // ---------------------------------------------------------------------------
 
 template <bool kGroupK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Warps<kGroupK>::kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs a) {
     using L = Layout<kGroupK>;
+    using Wp = Warps<kGroupK>;
+    constexpr int kThreads = Wp::kThreads, kEpiWarps = Wp::kEpiWarps, kCols = Wp::kCols;
     constexpr int kStages = L::kStages;
     constexpr int kScaleSlots = L::kScaleSlots;
     constexpr uint32_t kOffStages = L::kOffStages, kOffBars = L::kOffBars, kOffMisc = L::kOffMisc;
@@ -452,7 +451,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     ring.empty0 = ring_empty0;
 
     if (warp < kCtrlWarps) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Wp::kCtrlRegs));
       if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
@@ -565,10 +564,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Wp::kEpiRegs));
         // ---------------------------------------------------- promotion + epilogue
         const int ep = warp - kCtrlWarps;
-        const int half = ep >> 2;            // 128-column half of the tile
+        const int grp = ep >> 2;             // kCols-column group of the tile
         const int quarter = warp & 3;        // TMEM lane quarter this warp may access
         const int r = 32 * quarter + lane;   // tile row owned by this thread (row-grouped)
         const int g4 = lane >> 2, c2 = 2 * (lane & 3);   // 16x256b position (contraction-grouped)
@@ -588,9 +587,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             } else if ((tile += gridDim.x) >= total) {
                 break;
             }
-            float2 acc[64];   // columns 2i, 2i + 1 of this thread's 128-column half
+            float2 acc[kCols / 2];   // row-grouped: columns 2i, 2i + 1 of this thread's group
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < kCols / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             // Only what the K loop and the epilogue need stays live (registers
             // are the promotion's limit); output rows fit in 32 bits (checked
             // on the host).
@@ -603,7 +602,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 rows_valid = BM;
                 out_row0 = v.y;
                 row_ok = true;
-                col0 = v.z + 128 * half;
+                col0 = v.z + kCols * grp;
                 col_ok = col0 < a.N;
                 sa_p = sb_p = nullptr;
             } else {
@@ -612,25 +611,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 rows_valid = T.rows_valid;
                 out_row0 = (int)T.out_row0;
                 row_ok = r < T.rows_valid;
-                col0 = T.n0 + 128 * half;
+                col0 = T.n0 + kCols * grp;
                 col_ok = col0 < a.N;
                 sa_p = a.sa + T.rowA + r;
                 sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
             }
-            // row-grouped mode: the scales of the next K block are loaded while
-            // this one is promoted
-            float sa_n = 0.f, sb_n = 0.f;
+            // row-grouped mode: the scales of K block kb + 2 are loaded while kb
+            // is promoted
+            float sa_c = 0.f, sa_n = 0.f, sb_c = 0.f, sb_n = 0.f;
             if (!kGroupK) {
-                if (row_ok && nkb > 0) sa_n = __ldg(sa_p);
-                if (col_ok && nkb > 0) sb_n = __ldg(sb_p);
+                if (row_ok && nkb > 0) sa_c = __ldg(sa_p);
+                if (row_ok && nkb > 1) sa_n = __ldg(sa_p + a.M_total);
+                if (col_ok && nkb > 0) sb_c = __ldg(sb_p);
+                if (col_ok && nkb > 1) sb_n = __ldg(sb_p + 1);
             }
             for (int kb = 0; kb < nkb; ++kb) {
                 float s = 0.f;
                 if (!kGroupK) {
-                    s = sa_n * sb_n;
-                    if (kb + 1 < nkb) {
-                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 1) * a.M_total);
-                        if (col_ok) sb_n = __ldg(sb_p + kb + 1);
+                    s = sa_c * sb_c;
+                    sa_c = sa_n;
+                    sb_c = sb_n;
+                    if (kb + 2 < nkb) {
+                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 2) * a.M_total);
+                        if (col_ok) sb_n = __ldg(sb_p + kb + 2);
                     }
                 }
                 if (!mbar_wait(tfull_bar(buf), bphase, abort_flag, a.status)) {
@@ -639,11 +642,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 tc_fence_after();
                 const uint32_t taddr =
-                    tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * BN + 128 * half;
+                    tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * BN + kCols * grp;
                 if (!kGroupK) {
                     const float2 s2 = make_float2(s, s);
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
+                    for (int ch = 0; ch < kCols / 64; ++ch) {
                         uint32_t p[64];
                         tmem_ld64(taddr + 64 * ch, p);
 #pragma unroll
@@ -666,7 +669,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     float sak[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) sak[k] = slot[32 * quarter + g4 + 8 * k];
-                    const float* sbp = slot + BM + 128 * half + c2;
+                    const float* sbp = slot + BM + kCols * grp + c2;
 #pragma unroll
                     for (int cg = 0; cg < 2; ++cg) {
                         float2 sb2[8];
@@ -753,7 +756,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (a.out_f32) {
                     float* ob = static_cast<float*>(a.out) + col0 + 4 * quad;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
+                    for (int ch = 0; ch < kCols / 16; ++ch) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             my_row[q] = make_uint4(__float_as_uint(acc[8 * ch + 2 * q].x),
@@ -773,7 +776,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 } else {
                     uint16_t* ob = static_cast<uint16_t*>(a.out) + col0 + 8 * quad;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
+                    for (int ch = 0; ch < kCols / 32; ++ch) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             my_row[q] = make_uint4(pack_bf16x2(acc[16 * ch + 4 * q + 0].x, acc[16 * ch + 4 * q + 0].y),
@@ -890,7 +893,9 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     // the warpgroup register split must fit in what the CTA is launched with
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, (const void*)kern) != cudaSuccess) return FG8_ERR_CUDA;
-    if (fa.numRegs < kLaunchRegs) return FG8_ERR_UNSUPPORTED;
+    const int launch_regs = group_mode == FG8_GROUP_K ? Warps<true>::kLaunchRegs : Warps<false>::kLaunchRegs;
+    const int threads = group_mode == FG8_GROUP_K ? Warps<true>::kThreads : Warps<false>::kThreads;
+    if (fa.numRegs < launch_regs) return FG8_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes) !=
         cudaSuccess)
         return FG8_ERR_CUDA;
@@ -914,6 +919,6 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     int64_t grid = fg8h::num_sms();
     if (grid > max_tiles) grid = max_tiles;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, kThreads, smem_bytes, (cudaStream_t)stream>>>(mA, mB, mOut, args);
+    kern<<<(unsigned)grid, threads, smem_bytes, (cudaStream_t)stream>>>(mA, mB, mOut, args);
     return fg8h::launch_status();
 }
