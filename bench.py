@@ -290,16 +290,27 @@ class Step:
             fg8.FG8_BSCALE_ROW128, fg8.FG8_OUT_F32, self.dw, self.status, sp)))
         self.launches_per_step = n[0]
 
-    # host-side inputs / outputs of the end-to-end measurement
-    def host_io(self):
+    # --- end-to-end measurement: step inputs arrive from pinned host memory and
+    # the forward output and dX go back.  Inputs and those outputs have two
+    # device slots, so the copies of one step overlap the kernels of the next.
+    IN_NAMES = ("x", "ids", "dy", "h")
+
+    def out_names(self):
+        return ("y_dn" if self.h is not None else "y_up", "dx")
+
+    def make_slots(self):
+        names = [n for n in self.IN_NAMES if getattr(self, n) is not None] + list(self.out_names())
+        self.slots = [{n: getattr(self, n) for n in names},
+                      {n: torch.empty_like(getattr(self, n)) for n in names}]
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-        ins = [(pin(self.x), self.x), (pin(self.ids), self.ids), (pin(self.dy), self.dy)]
-        if self.h is not None:
-            ins.append((pin(self.h), self.h))
-        res = self.y_dn if self.h is not None else self.y_up
-        outs = [(torch.empty(res.shape, dtype=res.dtype).pin_memory(), res),
-                (torch.empty(self.dx.shape, dtype=self.dx.dtype).pin_memory(), self.dx)]
+        ins = {n: pin(getattr(self, n)) for n in self.IN_NAMES if getattr(self, n) is not None}
+        outs = {n: torch.empty(getattr(self, n).shape, dtype=getattr(self, n).dtype).pin_memory()
+                for n in self.out_names()}
         return ins, outs
+
+    def use_slot(self, i):
+        for n, t in self.slots[i].items():
+            setattr(self, n, t)
 
 
 # --------------------------------------------------------------------------
@@ -552,25 +563,54 @@ def main():
         gemm_tflops, quant_gbs = float(t[0]), float(t[1])
 
     # ---------------- end-to-end through the C ABI with host buffers
+    # Step i uses device slot i % 2: its inputs are copied in on one copy stream
+    # (once step i - 2 is done with the slot), the kernels run on the compute
+    # stream, and the forward output and dX go back on another copy stream, so
+    # host transfers in both directions overlap the kernels of the next step.
     e2e = None
     if not args.no_e2e:
-        ins, outs = st.host_io()
-        h2d = sum(h.numel() * h.element_size() for h, _ in ins)
-        d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+        host_in, host_out = st.make_slots()
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        comp_done, out_done = [None, None], [None, None]
         if pg:
             pg.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(args.steps):
-                for h, d in ins:
-                    d.copy_(h, non_blocking=True)
-                st.run(stream)
-                for h, d in outs:
-                    h.copy_(d, non_blocking=True)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(args.steps):
+            slot = i % 2
+            dev_slot = st.slots[slot]
+            in_done = ev()
+            with torch.cuda.stream(s_in):
+                if comp_done[slot] is not None:
+                    s_in.wait_event(comp_done[slot])
+                for n, h in host_in.items():
+                    dev_slot[n].copy_(h, non_blocking=True)
+                in_done.record(s_in)
+            stream.wait_event(in_done)
+            if out_done[slot] is not None:
+                stream.wait_event(out_done[slot])
+            st.use_slot(slot)
+            st.run(stream)
+            comp_done[slot] = ev()
+            comp_done[slot].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[slot])
+                for n, h in host_out.items():
+                    h.copy_(dev_slot[n], non_blocking=True)
+                out_done[slot] = ev()
+                out_done[slot].record(s_out)
+        for d in out_done:
+            if d is not None:
+                stream.wait_event(d)
         e1.record(stream)
         torch.cuda.synchronize()
+        st.use_slot(0)
         e2e_ms = e0.elapsed_time(e1) / args.steps
         if pg:
             t = torch.tensor([e2e_ms], device=dev)
@@ -579,7 +619,8 @@ def main():
         e2e = {"value": world * gemm_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "GEMM FLOPs per step over the whole step time including pinned-host "
-                       "copies of X, ids, H, dY in and the forward output and dX out"}
+                       "copies of X, ids, H, dY in and the forward output and dX out; two "
+                       "device slots, copies overlap the next step's kernels"}
     if st.status.item() != 0:
         raise RuntimeError(f"device status {fg8.status_name(st.status.item())}")
 

@@ -616,24 +616,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 sa_p = a.sa + T.rowA + r;
                 sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
             }
-            // row-grouped mode: the scales of K block kb + 2 are loaded while kb
-            // is promoted
-            float sa_c = 0.f, sa_n = 0.f, sb_c = 0.f, sb_n = 0.f;
+            // row-grouped mode: the scales of the next K block are loaded while
+            // this one is promoted (two blocks ahead measured slower in the full
+            // step: it costs the promotion a spilled register)
+            float sa_n = 0.f, sb_n = 0.f;
             if (!kGroupK) {
-                if (row_ok && nkb > 0) sa_c = __ldg(sa_p);
-                if (row_ok && nkb > 1) sa_n = __ldg(sa_p + a.M_total);
-                if (col_ok && nkb > 0) sb_c = __ldg(sb_p);
-                if (col_ok && nkb > 1) sb_n = __ldg(sb_p + 1);
+                if (row_ok && nkb > 0) sa_n = __ldg(sa_p);
+                if (col_ok && nkb > 0) sb_n = __ldg(sb_p);
             }
             for (int kb = 0; kb < nkb; ++kb) {
                 float s = 0.f;
                 if (!kGroupK) {
-                    s = sa_c * sb_c;
-                    sa_c = sa_n;
-                    sb_c = sb_n;
-                    if (kb + 2 < nkb) {
-                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 2) * a.M_total);
-                        if (col_ok) sb_n = __ldg(sb_p + kb + 2);
+                    s = sa_n * sb_n;
+                    if (kb + 1 < nkb) {
+                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 1) * a.M_total);
+                        if (col_ok) sb_n = __ldg(sb_p + kb + 1);
                     }
                 }
                 if (!mbar_wait(tfull_bar(buf), bphase, abort_flag, a.status)) {
