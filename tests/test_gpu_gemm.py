@@ -278,3 +278,66 @@ def test_gemm_kgrouped_dsv3_wgrad_full_size_sampled(oracle):
         if counts[e] == 0:
             assert np.all(got == 0)
         check(got.ravel(), ref, bound, f"wgrad expert {e}")
+
+
+def _kgrouped_operands(counts, M, N, seed):
+    counts = np.asarray(counts)
+    padoff = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]).astype(np.int32)
+    P = fg8.fg8_colwise_capacity(int(counts.sum()), len(counts))
+    a = W.gen_e4m3_codes((M, P), seed, 1)
+    b = W.gen_e4m3_codes((N, P), seed, 2)
+    sa = W.gen_scales((P // 128, M), seed, 3)
+    sb = W.gen_scales((P // 128, N), seed, 4)
+    return padoff, a, b, sa, sb
+
+
+def test_gemm_kgrouped_interleaved_order_full(oracle):
+    """Contraction-grouped with E divisible by 4, so tiles of four experts of
+    different sizes are interleaved at run time: 8 experts (two empty, one with
+    five K blocks), every output entry against the oracle."""
+    counts = [0, 700, 1, 130, 0, 64, 390, 128]
+    M, N, E = 256, 512, len(counts)
+    padoff, a, b, sa, sb = _kgrouped_operands(counts, M, N, 31)
+    st = fg8.new_status()
+    out = fg8.grouped_gemm(a.cuda(), sa.cuda(), b.cuda(), sb.cuda(), torch.from_numpy(padoff).cuda(),
+                           out_dtype=fg8.FG8_OUT_F32, group_mode=fg8.FG8_GROUP_K, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    got = out.cpu().numpy()
+    m, n = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+    for e in range(E):
+        ref, bound = oracle.gemm_kgrouped_entries(a.numpy(), sa.numpy(), b.numpy(), sb.numpy(),
+                                                  padoff, np.full(m.size, e), m.ravel(), n.ravel())
+        if counts[e] == 0:
+            assert np.all(got[e] == 0)
+        check(got[e].ravel(), ref, bound, f"interleaved expert {e}")
+
+
+def test_gemm_kgrouped_tile_counters_reused_and_concurrent():
+    """The contraction-grouped GEMM hands out tiles from library-held counters
+    (64, used in turn).  70 launches on one stream wrap around them, and pairs
+    of launches on two streams run at the same time; every result must equal
+    the first bit for bit (the kernel is deterministic)."""
+    counts = [5, 300, 0, 129, 77, 256, 1, 40]
+    M, N = 128, 256
+    padoff, a, b, sa, sb = _kgrouped_operands(counts, M, N, 33)
+    args = [t.cuda() for t in (a, sa, b, sb)] + [torch.from_numpy(padoff).cuda()]
+    st = fg8.new_status()
+
+    def run(stream=None):
+        return fg8.grouped_gemm(*args, out_dtype=fg8.FG8_OUT_F32, group_mode=fg8.FG8_GROUP_K,
+                                dev_status=st, stream=stream)
+
+    first = run()
+    torch.cuda.synchronize()
+    outs = [run() for _ in range(70)]
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(4):
+        with torch.cuda.stream(s1):
+            outs.append(run(s1.cuda_stream))
+        with torch.cuda.stream(s2):
+            outs.append(run(s2.cuda_stream))
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for o in outs:
+        assert torch.equal(o, first)

@@ -346,3 +346,26 @@ def test_transpose_blockq_dsv3_full_size_sampled(oracle):
         rT, _ = oracle.transpose_blockq(src, np.ones((1, 1, 1), np.float32))
         got = wqT[e, kb * 128:(kb + 1) * 128, nb * 128:(nb + 1) * 128].cpu().numpy()
         assert np.array_equal(got, rT[0]), (e, nb, kb)
+
+
+def test_quantize_rows_ragged_row_count(oracle):
+    """Identity mode with a row count that is not a multiple of the 128-row
+    boxes (the last box reads past the end as zeros) and three column tiles."""
+    x = W.gen_normal_bf16((300, 384), 1.0, 41, 1)
+    xq, sa = fg8.quantize_act_rows(x.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.quantize_act(x, None, 1)
+    assert np.array_equal(xq.cpu().numpy(), ref["xq"])
+    assert np.array_equal(sa.cpu().numpy(), ref["sa"])
+
+
+def test_quantize_weight_reports_ok_status(oracle):
+    """With a status word, a normal launch leaves it at FG8_OK."""
+    w = W.gen_normal_bf16((3, 256, 384), 0.02, 43, 1)
+    st = fg8.new_status()
+    wq, sw = fg8.quantize_weight(w.cuda(), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    rwq, rsw = oracle.quantize_weight(w)
+    assert np.array_equal(wq.cpu().numpy(), rwq)
+    assert np.array_equal(sw.cpu().numpy(), rsw)
