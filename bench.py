@@ -98,9 +98,11 @@ def work_of(cfg: W.MoEConfig, padded_total: int):
     T, K, k, E, R, N, I = cfg.T, cfg.hidden, cfg.k, cfg.E, cfg.R, cfg.n_up, cfg.inter
     w = {
         "quant_act_permute": ("hbm", bytes_route_quant(T, K, k, E)),
-        "quant_weight": ("hbm", bytes_weight_quant(E, N, K) + (bytes_weight_quant(E, K, I) if I else 0)),
+        # up weight: quantized with its block-transposed copy written in the same
+        # pass (one more byte per element and a scale per block)
+        "quant_weight": ("hbm", bytes_weight_quant(E, N, K) + E * N * K + 4 * E * (N // 128) * (K // 128)
+                         + (bytes_weight_quant(E, K, I) if I else 0)),
         "gemm_fprop_up": ("tensor", 2 * R * N * K),
-        "transpose_blockq": ("hbm", bytes_transpose(E, N, K)),
         "quant_act_rows": ("hbm", bytes_rows_quant(R, N) + (bytes_rows_quant(R, I) if I else 0)),
         "gemm_dgrad": ("tensor", 2 * R * K * N),
         "quant_act_colwise": ("hbm", bytes_colwise(R, N, padded_total) + bytes_colwise(T, K, padded_total)),
@@ -151,6 +153,14 @@ def source_hash(group: str) -> str:
     return h.hexdigest()[:12]
 
 
+def algorithmic_bytes(family: str, cfg: W.MoEConfig, padded_total: int) -> float:
+    """The bytes a family must move on `cfg` (GEMMs: operands + output once)."""
+    if family == "transpose_blockq":
+        return bytes_transpose(cfg.E, cfg.n_up, cfg.hidden)
+    w, gb = work_of(cfg, padded_total)
+    return gb.get(family, w[family][1])
+
+
 def measured_traffic(family: str, cfg: W.MoEConfig, padded_total: int):
     entry = TRAFFIC_CAPTURE["families"].get(family)
     if entry is None:
@@ -159,11 +169,8 @@ def measured_traffic(family: str, cfg: W.MoEConfig, padded_total: int):
     if source_hash(group) != sha:
         return None
     cap = W.CONFIGS[TRAFFIC_CAPTURE["config"]]
-    w_cap, gb_cap = work_of(cap, padded_total_of(cap))
-    w_now, gb_now = work_of(cfg, padded_total)
-    num = gb_now.get(family, w_now[family][1])
-    den = gb_cap.get(family, w_cap[family][1])
-    return bytes_cap * num / den
+    return bytes_cap * algorithmic_bytes(family, cfg, padded_total) / \
+        algorithmic_bytes(family, cap, padded_total_of(cap))
 
 
 # --------------------------------------------------------------------------
@@ -246,7 +253,8 @@ class Step:
             self.status, sp)))
 
         def wquant():
-            fg8.fg8_quantize_weight(u16(self.w_up), E, N, K, self.wq_up, self.sw_up, self.status, sp)
+            fg8.fg8_quantize_weight_transposed(u16(self.w_up), E, N, K, self.wq_up, self.sw_up,
+                                               self.wqT_up, self.swT_up, self.status, sp)
             n[0] += 1
             if I:
                 fg8.fg8_quantize_weight(u16(self.w_down), E, K, I, self.wq_dn, self.sw_dn, self.status, sp)
@@ -270,8 +278,6 @@ class Step:
                 self.hq, self.sh, self.wq_dn, self.sw_dn, self.offsets, R, K, I, E,
                 fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_dn,
                 self.status, sp)))
-        timed("transpose_blockq", launch(lambda: fg8.fg8_transpose_blockq(
-            self.wq_up, self.sw_up, E, N, K, self.wqT_up, self.swT_up, sp)))
         timed("gemm_dgrad", launch(lambda: fg8.fg8_grouped_gemm(
             self.dyq, self.sdy, self.wqT_up, self.swT_up, self.offsets, R, K, N, E,
             fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.dx, self.status, sp)))
@@ -289,6 +295,14 @@ class Step:
             self.dyT, self.sdyT, self.xT, self.sxT, self.pad_dy, N, K, self.P, E, fg8.FG8_GROUP_K,
             fg8.FG8_BSCALE_ROW128, fg8.FG8_OUT_F32, self.dw, self.status, sp)))
         self.launches_per_step = n[0]
+
+    def run_transpose(self, stream):
+        """The standalone block transpose (fg8_transpose_blockq) of the up
+        weight: the step gets WqT from the fused quantizer, this times the
+        transpose kernel on its own, outside the step."""
+        c = self.cfg
+        self.fg8.fg8_transpose_blockq(self.wq_up, self.sw_up, c.E, c.n_up, c.hidden, self.wqT_up,
+                                      self.swT_up, stream.cuda_stream)
 
     # --- end-to-end measurement: step inputs arrive from pinned host memory and
     # the forward output and dX go back.  Inputs and those outputs have two
@@ -555,6 +569,23 @@ def main():
         entry["traffic"] = measured_traffic(name, cfg, st.padded_total)
         kernels.append(entry)
     dom = max(kernels, key=lambda d: d["ms"])
+    # K3 on its own (the step takes WqT from the fused quantizer): timed with
+    # events around args.steps back-to-back launches, outside the step
+    with torch.cuda.stream(stream):
+        st.run_transpose(stream)
+        tr0, tr1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tr0.record(stream)
+        for _ in range(args.steps):
+            st.run_transpose(stream)
+        tr1.record(stream)
+    torch.cuda.synchronize()
+    tr_ms = tr0.elapsed_time(tr1) / args.steps
+    tr_gb = bytes_transpose(cfg.E, cfg.n_up, cfg.hidden) / (tr_ms * 1e-3) / 1e9
+    kernels.append({"kernel": "transpose_blockq", "standalone": True, "bound": "hbm", "ms": tr_ms,
+                    "achieved": tr_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": tr_gb / pk["hbm_gbs"], "share": None,
+                    "traffic": measured_traffic("transpose_blockq", cfg, st.padded_total),
+                    "note": "not in the step: the step's WqT comes from the fused quantizer"})
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
     quant_gbs = q_bytes / (q_ms * 1e-3) / 1e9
     if pg:

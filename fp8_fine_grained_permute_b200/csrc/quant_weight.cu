@@ -25,10 +25,19 @@ using namespace fg8::tma;
 constexpr int kThreads = 256;
 constexpr uint32_t kBlockBytes = 128 * 256;   // bf16 128 x 128
 
-__global__ void __launch_bounds__(kThreads, 5)
+// word w of code row r sits at word w ^ swz(r) of the shared code tile: conflict
+// free both for the row-wise writes and for the transposed reads below
+__device__ __forceinline__ int swz(int r) { return ((r >> 2) ^ (r & 3)) & 31; }
+
+// kT: also write the block-transposed copy (wqT[e][k][n] = wq[e][n][k],
+// swT[e][kb][nb] = sw[e][nb][kb]) from the codes still in shared memory, so
+// the backward pass's copy costs no second read of wq.
+template <bool kT>
+__global__ void __launch_bounds__(kThreads, kT ? 4 : 5)
 quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t K,
-                    uint8_t* __restrict__ wq, float* __restrict__ sw, int32_t* status) {
-    extern __shared__ __align__(128) uint8_t blk[];   // [128 rows][256 bytes]
+                    uint8_t* __restrict__ wq, float* __restrict__ sw, uint8_t* __restrict__ wqT,
+                    float* __restrict__ swT, int32_t* status) {
+    extern __shared__ __align__(128) uint8_t blk[];   // [128 rows][256 bytes] (+ code tile)
     __shared__ __align__(8) uint64_t bar;
     __shared__ float red[kThreads / 32];
     __shared__ int abort_flag;
@@ -64,12 +73,69 @@ quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t 
     const fg8::QScale q = fg8::make_qscale(s);
     const int64_t base = ((int64_t)e * N + (int64_t)nb * 128) * K + (int64_t)kb * 128;
     uint8_t* dst = wq + base + chunk * 8;
+    uint32_t* codes = reinterpret_cast<uint32_t*>(blk + kBlockBytes);   // [128][32] words (kT)
 #pragma unroll 2
     for (int i = 0; i < 8; ++i) {
-        const uint4 v = *reinterpret_cast<const uint4*>(blk + (r0 + 16 * i) * 256 + chunk * 16);
-        *reinterpret_cast<uint2*>(dst + (int64_t)(r0 + 16 * i) * K) = fg8::quant8(v, q);
+        const int r = r0 + 16 * i;
+        const uint4 v = *reinterpret_cast<const uint4*>(blk + r * 256 + chunk * 16);
+        const uint2 c = fg8::quant8(v, q);
+        *reinterpret_cast<uint2*>(dst + (int64_t)r * K) = c;
+        if (kT) {
+            codes[r * 32 + ((2 * chunk) ^ swz(r))] = c.x;
+            codes[r * 32 + ((2 * chunk + 1) ^ swz(r))] = c.y;
+        }
     }
-    if (t == 0) sw[((int64_t)e * NB + nb) * KB + kb] = ok ? s : __int_as_float(0x7FC00000);
+    const float s_out = ok ? s : __int_as_float(0x7FC00000);
+    if (t == 0) sw[((int64_t)e * NB + nb) * KB + kb] = s_out;
+    if (kT) {
+        __syncthreads();
+        // lane i of the warp on word column j reads words j of code rows
+        // 4i..4i+3, transposes the 4x4 bytes and writes word i of output rows
+        // 4j..4j+3: each warp store is one 128-byte output row segment
+        const int lane = t & 31, warp = t >> 5;
+        uint8_t* dT = wqT + ((int64_t)e * K + (int64_t)kb * 128) * N + (int64_t)nb * 128;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = warp + 8 * jj;
+            const uint32_t a0 = codes[(4 * lane + 0) * 32 + (j ^ swz(4 * lane + 0))];
+            const uint32_t a1 = codes[(4 * lane + 1) * 32 + (j ^ swz(4 * lane + 1))];
+            const uint32_t a2 = codes[(4 * lane + 2) * 32 + (j ^ swz(4 * lane + 2))];
+            const uint32_t a3 = codes[(4 * lane + 3) * 32 + (j ^ swz(4 * lane + 3))];
+            const uint32_t t0 = __byte_perm(a0, a1, 0x5140), t1 = __byte_perm(a2, a3, 0x5140);
+            const uint32_t t2 = __byte_perm(a0, a1, 0x7362), t3 = __byte_perm(a2, a3, 0x7362);
+            uint32_t* d = reinterpret_cast<uint32_t*>(dT + (int64_t)(4 * j) * N) + lane;
+            d[0] = __byte_perm(t0, t1, 0x5410);
+            d[N / 4] = __byte_perm(t0, t1, 0x7632);
+            d[2 * (N / 4)] = __byte_perm(t2, t3, 0x5410);
+            d[3 * (N / 4)] = __byte_perm(t2, t3, 0x7632);
+        }
+        if (t == 0) swT[((int64_t)e * KB + kb) * NB + nb] = s_out;
+    }
+}
+
+fg8_status launch(const uint16_t* w, int E, int N, int K, uint8_t* wq, float* sw, uint8_t* wqT,
+                  float* swT, int32_t* dev_status, cudaStream_t stream) {
+    if (!w || !wq || !sw) return FG8_ERR_INVALID_ARG;
+    if (E < 1 || N < 128 || K < 128 || N % 128 || K % 128) return FG8_ERR_INVALID_ARG;
+    if (N / 128 > 65535 || E > 65535) return FG8_ERR_UNSUPPORTED;
+    if (!fg8h::aligned16(w) || !fg8h::aligned16(wq) || (reinterpret_cast<uintptr_t>(sw) & 3) ||
+        (reinterpret_cast<uintptr_t>(dev_status) & 3))
+        return FG8_ERR_INVALID_ARG;
+    const bool tr = wqT != nullptr;
+    if (tr && (!swT || !fg8h::aligned16(wqT) || (reinterpret_cast<uintptr_t>(swT) & 3)))
+        return FG8_ERR_INVALID_ARG;
+    CUtensorMap m;
+    if (!fg8h::make_tensor_map_2d(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, (uint64_t)E * N,
+                                  (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return FG8_ERR_CUDA;
+    auto kern = tr ? quant_weight_blocks<true> : quant_weight_blocks<false>;
+    const uint32_t smem = kBlockBytes + (tr ? 128 * 128 : 0);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return FG8_ERR_CUDA;
+    dim3 grid(K / 128, N / 128, E);
+    kern<<<grid, kThreads, smem, stream>>>(m, N, K, wq, sw, wqT, swT, dev_status);
+    return fg8h::launch_status();
 }
 
 }  // namespace
@@ -77,21 +143,13 @@ quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t 
 extern "C" fg8_status fg8_quantize_weight(const uint16_t* w, int E, int N, int K,
                                           uint8_t* wq, float* sw, int32_t* dev_status,
                                           fg8_stream_t stream) {
-    if (!w || !wq || !sw) return FG8_ERR_INVALID_ARG;
-    if (E < 1 || N < 128 || K < 128 || N % 128 || K % 128) return FG8_ERR_INVALID_ARG;
-    if (N / 128 > 65535 || E > 65535) return FG8_ERR_UNSUPPORTED;
-    if (!fg8h::aligned16(w) || !fg8h::aligned16(wq) || (reinterpret_cast<uintptr_t>(sw) & 3) ||
-        (reinterpret_cast<uintptr_t>(dev_status) & 3))
-        return FG8_ERR_INVALID_ARG;
-    CUtensorMap m;
-    if (!fg8h::make_tensor_map_2d(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, (uint64_t)E * N,
-                                  (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return FG8_ERR_CUDA;
-    if (cudaFuncSetAttribute(quant_weight_blocks, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kBlockBytes) != cudaSuccess)
-        return FG8_ERR_CUDA;
-    dim3 grid(K / 128, N / 128, E);
-    quant_weight_blocks<<<grid, kThreads, kBlockBytes, (cudaStream_t)stream>>>(m, N, K, wq, sw,
-                                                                               dev_status);
-    return fg8h::launch_status();
+    return launch(w, E, N, K, wq, sw, nullptr, nullptr, dev_status, (cudaStream_t)stream);
+}
+
+extern "C" fg8_status fg8_quantize_weight_transposed(const uint16_t* w, int E, int N, int K,
+                                                     uint8_t* wq, float* sw, uint8_t* wqT,
+                                                     float* swT, int32_t* dev_status,
+                                                     fg8_stream_t stream) {
+    if (!wqT || !swT) return FG8_ERR_INVALID_ARG;
+    return launch(w, E, N, K, wq, sw, wqT, swT, dev_status, (cudaStream_t)stream);
 }

@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.fg8_colwise_capacity.argtypes = [_I64, _I]
         L.fg8_quantize_weight.restype = _I
         L.fg8_quantize_weight.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P]
+        L.fg8_quantize_weight_transposed.restype = _I
+        L.fg8_quantize_weight_transposed.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P]
         L.fg8_transpose_blockq.restype = _I
         L.fg8_transpose_blockq.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P]
         L.fg8_grouped_gemm.restype = _I
@@ -147,6 +149,12 @@ def fg8_quantize_act_workspace(T: int, k: int, E: int) -> int:
 
 def fg8_colwise_capacity(R: int, E: int) -> int:
     return lib().fg8_colwise_capacity(R, E)
+
+
+def fg8_quantize_weight_transposed(w, E, N, K, wq, sw, wqT, swT, dev_status=None, stream=None):
+    _check(lib().fg8_quantize_weight_transposed(_ptr(w), E, N, K, _ptr(wq), _ptr(sw), _ptr(wqT),
+                                                _ptr(swT), _ptr(dev_status), _stream(stream)),
+           "fg8_quantize_weight_transposed")
 
 
 def fg8_quantize_weight(w, E, N, K, wq, sw, dev_status=None, stream=None):
@@ -251,6 +259,18 @@ def quantize_weight(w: torch.Tensor, status=None, stream=None):
     sw = torch.empty((E, N // 128, K // 128), dtype=torch.float32, device=w.device)
     fg8_quantize_weight(_u16(w), E, N, K, wq, sw, status, stream)
     return wq, sw
+
+
+def quantize_weight_transposed(w: torch.Tensor, status=None, stream=None):
+    """128x128 block quantize of bf16 w [E,N,K] plus its block-transposed copy
+    -> (wq, sw, wqT [E,K,N], swT [E,K/128,N/128])."""
+    E, N, K = w.shape
+    wq = torch.empty((E, N, K), dtype=torch.uint8, device=w.device)
+    sw = torch.empty((E, N // 128, K // 128), dtype=torch.float32, device=w.device)
+    wqT = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
+    swT = torch.empty((E, K // 128, N // 128), dtype=torch.float32, device=w.device)
+    fg8_quantize_weight_transposed(_u16(w), E, N, K, wq, sw, wqT, swT, status, stream)
+    return wq, sw, wqT, swT
 
 
 def transpose_blockq(wq: torch.Tensor, sw: torch.Tensor, stream=None):

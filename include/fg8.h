@@ -161,6 +161,20 @@ fg8_status fg8_quantize_weight(const uint16_t* w, int E, int N, int K,
                                fg8_stream_t stream);
 
 /*
+ * fg8_quantize_weight_transposed -- fg8_quantize_weight that also writes the
+ * block-transposed copy the backward pass needs (the output of
+ * fg8_transpose_blockq) from the codes it has just formed, so producing both
+ * costs one read of w instead of an extra read of wq.  Outputs are identical
+ * to fg8_quantize_weight followed by fg8_transpose_blockq.
+ *   w, wq, sw, dev_status  as for fg8_quantize_weight
+ *   wqT  E4M3 [E][K][N], 16-byte aligned
+ *   swT  fp32 [E][K/128][N/128]
+ */
+fg8_status fg8_quantize_weight_transposed(const uint16_t* w, int E, int N, int K,
+                                          uint8_t* wq, float* sw, uint8_t* wqT, float* swT,
+                                          int32_t* dev_status, fg8_stream_t stream);
+
+/*
  * fg8_transpose_blockq -- transpose an already block-quantized weight and its
  * scale grid for backward, so only the forward FP8 copy is stored ([K2] FP8
  * paragraph, last sentence).  Pure byte/scale moves: because the blocks are

@@ -369,3 +369,34 @@ def test_quantize_weight_reports_ok_status(oracle):
     rwq, rsw = oracle.quantize_weight(w)
     assert np.array_equal(wq.cpu().numpy(), rwq)
     assert np.array_equal(sw.cpu().numpy(), rsw)
+
+
+@pytest.mark.parametrize("shape", [(3, 256, 384), (2, 512, 128)])
+def test_quantize_weight_transposed_matches_oracle(oracle, shape):
+    """The fused quantize + block transpose: wq, sw as fg8_quantize_weight,
+    wqT, swT as the oracle's transpose of the oracle's quantization."""
+    w = W.gen_normal_bf16(shape, 0.02, 47, 1)
+    st = fg8.new_status()
+    wq, sw, wqT, swT = fg8.quantize_weight_transposed(w.cuda(), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    rwq, rsw = oracle.quantize_weight(w)
+    rwqT, rswT = oracle.transpose_blockq(rwq, rsw)
+    assert np.array_equal(wq.cpu().numpy(), rwq)
+    assert np.array_equal(sw.cpu().numpy(), rsw)
+    assert np.array_equal(wqT.cpu().numpy(), rwqT)
+    assert np.array_equal(swT.cpu().numpy(), rswT)
+
+
+def test_quantize_weight_transposed_dsv3_up_equals_separate_kernels():
+    """At the DeepSeek-V3 up-projection size the fused kernel's transposed copy
+    equals fg8_transpose_blockq applied to its forward copy, byte for byte."""
+    cfg = W.CONFIGS["dsv3"]
+    w = W.gen_w_up(cfg, "cuda")
+    wq, sw, wqT, swT = fg8.quantize_weight_transposed(w)
+    wq2, sw2 = fg8.quantize_weight(w)
+    assert torch.equal(wq, wq2) and torch.equal(sw, sw2)
+    del w, wq2, sw2
+    wqT2, swT2 = fg8.transpose_blockq(wq, sw)
+    torch.cuda.synchronize()
+    assert torch.equal(wqT, wqT2) and torch.equal(swT, swT2)
