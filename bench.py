@@ -129,14 +129,14 @@ TRAFFIC_CAPTURE = {
     "config": "kanana",
     "families": {
         "quant_act_permute": (224.8e6, "quant_act", "20970841eab1"),
-        "quant_weight": (840.1e6, "quant_weight", "0c431cbcafdb"),
-        "gemm_fprop_up": (679.4e6, "gemm", "5b9d1343ec4e"),
-        "gemm_fprop_down": (529.6e6, "gemm", "5b9d1343ec4e"),
+        "quant_weight": (1026.8e6, "quant_weight", "9614c0fc5313"),
+        "gemm_fprop_up": (680.9e6, "gemm", "c4c6456bac63"),
+        "gemm_fprop_down": (530.8e6, "gemm", "c4c6456bac63"),
         "transpose_blockq": (345.9e6, "transpose", "c1e4961cfa8c"),
-        "quant_act_rows": (624.2e6, "quant_act", "20970841eab1"),
-        "gemm_dgrad": (721.7e6, "gemm", "5b9d1343ec4e"),
-        "quant_act_colwise": (663.4e6, "quant_act", "20970841eab1"),
-        "gemm_wgrad": (1150.7e6, "gemm", "5b9d1343ec4e"),
+        "quant_act_rows": (627.0e6, "quant_act", "20970841eab1"),
+        "gemm_dgrad": (722.5e6, "gemm", "c4c6456bac63"),
+        "quant_act_colwise": (664.7e6, "quant_act", "20970841eab1"),
+        "gemm_wgrad": (1151.7e6, "gemm", "c4c6456bac63"),
     },
 }
 _SRC = {"quant_act": ["quant_act.cu", "fg8_tma.cuh"], "quant_weight": ["quant_weight.cu", "fg8_tma.cuh"],
