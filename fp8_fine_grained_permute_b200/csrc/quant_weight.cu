@@ -33,11 +33,11 @@ __device__ __forceinline__ int swz(int r) { return ((r >> 2) ^ (r & 3)) & 31; }
 // swT[e][kb][nb] = sw[e][nb][kb]) from the codes still in shared memory, so
 // the backward pass's copy costs no second read of wq.
 template <bool kT>
-__global__ void __launch_bounds__(kThreads, kT ? 4 : 5)
+__global__ void __launch_bounds__(kThreads, 5)
 quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t K,
                     uint8_t* __restrict__ wq, float* __restrict__ sw, uint8_t* __restrict__ wqT,
                     float* __restrict__ swT, int32_t* status) {
-    extern __shared__ __align__(128) uint8_t blk[];   // [128 rows][256 bytes] (+ code tile)
+    extern __shared__ __align__(128) uint8_t blk[];   // [128 rows][256 bytes]
     __shared__ __align__(8) uint64_t bar;
     __shared__ float red[kThreads / 32];
     __shared__ int abort_flag;
@@ -73,7 +73,11 @@ quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t 
     const fg8::QScale q = fg8::make_qscale(s);
     const int64_t base = ((int64_t)e * N + (int64_t)nb * 128) * K + (int64_t)kb * 128;
     uint8_t* dst = wq + base + chunk * 8;
-    uint32_t* codes = reinterpret_cast<uint32_t*>(blk + kBlockBytes);   // [128][32] words (kT)
+    // kT: code row r (128 bytes) goes into the first half of bf16 row r's own
+    // bytes.  Row r is read only by the 16 lanes that write its codes (two
+    // rows per warp), so a warp barrier between the reads and the writes is
+    // enough, and no second tile is needed.
+    uint32_t* codes = reinterpret_cast<uint32_t*>(blk);   // row r at word 64 r
 #pragma unroll 2
     for (int i = 0; i < 8; ++i) {
         const int r = r0 + 16 * i;
@@ -81,8 +85,9 @@ quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t 
         const uint2 c = fg8::quant8(v, q);
         *reinterpret_cast<uint2*>(dst + (int64_t)r * K) = c;
         if (kT) {
-            codes[r * 32 + ((2 * chunk) ^ swz(r))] = c.x;
-            codes[r * 32 + ((2 * chunk + 1) ^ swz(r))] = c.y;
+            __syncwarp();
+            codes[r * 64 + ((2 * chunk) ^ swz(r))] = c.x;
+            codes[r * 64 + ((2 * chunk + 1) ^ swz(r))] = c.y;
         }
     }
     const float s_out = ok ? s : __int_as_float(0x7FC00000);
@@ -97,10 +102,10 @@ quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t 
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const int j = warp + 8 * jj;
-            const uint32_t a0 = codes[(4 * lane + 0) * 32 + (j ^ swz(4 * lane + 0))];
-            const uint32_t a1 = codes[(4 * lane + 1) * 32 + (j ^ swz(4 * lane + 1))];
-            const uint32_t a2 = codes[(4 * lane + 2) * 32 + (j ^ swz(4 * lane + 2))];
-            const uint32_t a3 = codes[(4 * lane + 3) * 32 + (j ^ swz(4 * lane + 3))];
+            const uint32_t a0 = codes[(4 * lane + 0) * 64 + (j ^ swz(4 * lane + 0))];
+            const uint32_t a1 = codes[(4 * lane + 1) * 64 + (j ^ swz(4 * lane + 1))];
+            const uint32_t a2 = codes[(4 * lane + 2) * 64 + (j ^ swz(4 * lane + 2))];
+            const uint32_t a3 = codes[(4 * lane + 3) * 64 + (j ^ swz(4 * lane + 3))];
             const uint32_t t0 = __byte_perm(a0, a1, 0x5140), t1 = __byte_perm(a2, a3, 0x5140);
             const uint32_t t2 = __byte_perm(a0, a1, 0x7362), t3 = __byte_perm(a2, a3, 0x7362);
             uint32_t* d = reinterpret_cast<uint32_t*>(dT + (int64_t)(4 * j) * N) + lane;
@@ -129,7 +134,7 @@ fg8_status launch(const uint16_t* w, int E, int N, int K, uint8_t* wq, float* sw
                                   (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
         return FG8_ERR_CUDA;
     auto kern = tr ? quant_weight_blocks<true> : quant_weight_blocks<false>;
-    const uint32_t smem = kBlockBytes + (tr ? 128 * 128 : 0);
+    const uint32_t smem = kBlockBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return FG8_ERR_CUDA;
