@@ -430,6 +430,25 @@ class OracleSample:
         return flops / t_gemm / 1e12, self.q_bytes / t_quant / 1e9, desc
 
 
+# --------------------------------------------------------------------------
+# replicas (one process per GPU, each running the whole step)
+# --------------------------------------------------------------------------
+
+def all_max(pg, values, device):
+    """Elementwise max over the ranks of `pg` (the values unchanged without one)."""
+    if pg is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(world: int, units_per_rank: float, slowest_ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed
+    `units_per_rank`: all units over the slowest rank's time (units/s)."""
+    return world * units_per_rank / (slowest_ms * 1e-3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -529,11 +548,7 @@ def main():
     if pg:
         pg.barrier()
     clocks = clk.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    (total_ms,) = all_max(pg, [t_start.elapsed_time(t_end)], dev)
     ms_step = total_ms / args.steps
     kern_ms = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in marks.items()}
 
@@ -586,12 +601,10 @@ def main():
                     "frac": tr_gb / pk["hbm_gbs"], "share": None,
                     "traffic": measured_traffic("transpose_blockq", cfg, st.padded_total),
                     "note": "not in the step: the step's WqT comes from the fused quantizer"})
-    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
-    quant_gbs = q_bytes / (q_ms * 1e-3) / 1e9
-    if pg:
-        t = torch.tensor([gemm_tflops, quant_gbs], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.SUM)
-        gemm_tflops, quant_gbs = float(t[0]), float(t[1])
+    # whole job: every rank did the same work; divide by the slowest rank's time
+    gemm_ms, q_ms = all_max(pg, [gemm_ms, q_ms], dev)
+    gemm_tflops = job_rate(world, gemm_flops, gemm_ms) / 1e12
+    quant_gbs = job_rate(world, q_bytes, q_ms) / 1e9
 
     # ---------------- end-to-end through the C ABI with host buffers
     # Step i uses device slot i % 2: its inputs are copied in on one copy stream
@@ -642,12 +655,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         st.use_slot(0)
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * gemm_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        (e2e_ms,) = all_max(pg, [e0.elapsed_time(e1) / args.steps], dev)
+        e2e = {"value": job_rate(world, gemm_flops, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "GEMM FLOPs per step over the whole step time including pinned-host "
                        "copies of X, ids, H, dY in and the forward output and dX out; two "
