@@ -283,15 +283,17 @@ struct ColArgs {
 // through row_map) are found once; then, for each column block in turn, the
 // 128 x 256-byte slice is brought into shared memory by cp.async (16 bytes a
 // thread-copy, padding rows zero-filled), two stages deep, so the next block's
-// data is in flight while this one is converted.  Thread t owns the column
-// pair p = t % 64 (columns 2p, 2p+1) for the 32 tokens of quarter q = t / 64:
-// it reads them as 32-bit words (a warp reads one 128-byte row piece,
-// conflict-free), reduces its two column maxima in registers (16-bit SIMD
-// max), and the four quarters of a pair combine through shared memory.  Codes
-// are then formed per column on 8 consecutive tokens at a time (bracketed
-// fast path) and stored transposed: 32 contiguous bytes (a whole sector) of
-// each column per thread.  (Measured against one CTA per 128 x 128 tile, with
-// the expert prefix recomputed by every CTA: 25% slower.)
+// data is in flight while this one is converted; one block barrier per column
+// block.  Warp wp owns the column pairs 8 wp .. 8 wp + 7, lane 8 q + pl the 32
+// tokens of quarter q of pair p = 8 wp + pl: it reads them as 32-bit words
+// (rows are stored XOR-swizzled by quarter, so the warp's reads hit 32 banks),
+// reduces its two column maxima in registers (16-bit SIMD max) and combines
+// the quarters with two shuffles.  Codes are then formed per column on 8
+// consecutive tokens at a time (bracketed fast path) and stored transposed:
+// 32 contiguous bytes (a whole sector) of each column per thread.  (Measured
+// against one CTA per 128 x 128 tile with the expert prefix recomputed by
+// every CTA: 25% slower; against the quarters combined through shared
+// memory with a second barrier: 4% slower.)
 constexpr uint32_t kColTileBytes = 128 * 256;
 constexpr int kColCtasPerSm = 3;
 constexpr int kColGroups = 4;      // column groups per tile (grid.y)
@@ -306,7 +308,6 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
     __shared__ int32_t s_pref[kMaxE + 1];
     __shared__ int32_t s_warp[33];
     __shared__ int32_t s_rows[128];
-    __shared__ uint32_t s_amax[2][4][64];
 
     const int t = threadIdx.x;
     const int E = a.E;
@@ -356,37 +357,39 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
         srcp[j] = a.x + (sr >= 0 ? (int64_t)sr * a.C + (u & 15) * 8 : 0);
         nbytes[j] = sr >= 0 ? 16u : 0u;
     }
+    // stage layout: word w of row r at word w ^ sw(r), sw(r) = 8 * ((r >> 5) & 3),
+    // so the four token quarters a warp reads land on different banks
     auto issue = [&](int cb, int st) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int u = t + kColThreads * j;
-            cp_async16(fg8::tma::smem_u32(s_tile + st * kColTileBytes + (u >> 4) * 256 + (u & 15) * 16),
+            const int row = u >> 4, ch = u & 15;
+            const int pw = (4 * ch) ^ (8 * ((row >> 5) & 3));
+            cp_async16(fg8::tma::smem_u32(s_tile + st * kColTileBytes + row * 256 + pw * 4),
                        srcp[j] + (nbytes[j] ? (int64_t)cb * 128 : 0), nbytes[j]);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    const int p = t & 63, q = t >> 6;
+    // warp wp owns column pairs 8 wp .. 8 wp + 7; lane = 8 q + pl: quarter q of
+    // the tokens (32 each) of pair p = 8 wp + pl
+    const int wp = t >> 5, lane = t & 31;
+    const int q = lane >> 3, p = 8 * wp + (lane & 7);
     if (cb0 < cb1) issue(cb0, 0);
     for (int cb = cb0; cb < cb1; ++cb) {
         const int st = (cb - cb0) & 1;
-        if (cb + 1 < cb1) {
-            issue(cb + 1, st ^ 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
-        __syncthreads();
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();   // this block of rows has landed; the other stage is free
+        if (cb + 1 < cb1) issue(cb + 1, st ^ 1);
         const int64_t col0 = (int64_t)cb * 128;
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(s_tile + st * kColTileBytes) + p;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(s_tile + st * kColTileBytes);
         uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = src[(32 * q + i) * 64];
+        for (int i = 0; i < 32; ++i) w[i] = src[(32 * q + i) * 64 + (p ^ (8 * q))];
         uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-        s_amax[st][q][p] = m;
-        __syncthreads();   // amax of this stage complete; also: every thread is done reading the other stage
-        m = __vmaxu2(__vmaxu2(s_amax[st][0][p], s_amax[st][1][p]), __vmaxu2(s_amax[st][2][p], s_amax[st][3][p]));
+        m = __vmaxu2(m, __shfl_xor_sync(kFull, m, 8));
+        m = __vmaxu2(m, __shfl_xor_sync(kFull, m, 16));
         const float s0 = fg8::tile_scale(__uint_as_float((m & 0xFFFFu) << 16));
         const float s1 = fg8::tile_scale(__uint_as_float(m & 0xFFFF0000u));
         const fg8::QScale q0 = fg8::make_qscale(s0), q1 = fg8::make_qscale(s1);
