@@ -107,17 +107,6 @@ FG8_DEV uint64_t mul_f32x2(uint64_t a, uint64_t b) {
     return d;
 }
 
-// E4M3 codes of (x0, x1) with scale context q, x0 in bits 7..0.
-FG8_DEV uint32_t quant_pair(float x0, float x1, const QScale& q) {
-    if (!q.exact) {
-        const uint64_t x = pack_f32x2(x0, x1);
-        const uint32_t lo = cvt_e4m3x2(mul_f32x2(x, pack_f32x2(q.r_lo, q.r_lo)));
-        const uint32_t hi = cvt_e4m3x2(mul_f32x2(x, pack_f32x2(q.r_hi, q.r_hi)));
-        if (lo == hi) return lo;
-    }
-    return cvt_e4m3x2(__fdiv_rn(x0, q.s), __fdiv_rn(x1, q.s));
-}
-
 // Fast-path codes of 8 bf16 values (one uint4): the codes of x * r(1 - eps)
 // and of x * r(1 + eps).  No branch, so callers can keep many of these in
 // flight and check them together (exact when lo == hi and !q.exact).
