@@ -42,56 +42,67 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Quantize one token row (K bf16, K % 128 == 0) in 1x128 tiles and store the
 // codes into the `nd` rows held by lanes 0..nd-1 of `my_row` (negative rows
-// are skipped).  The warp walks the row in 256-element segments: lane l holds
-// elements 8l..8l+7, lanes 0-15 form one tile and lanes 16-31 the next.
+// are skipped).  Eight lanes own one tile (16 values each: 16-byte chunks j and
+// j + 8, so a warp's loads are whole 128-byte lines), a warp four tiles at a
+// time, two such groups (eight tiles) in flight per iteration; the tile scale
+// is computed once per 16 values.
 __device__ __forceinline__ void quant_row(const uint16_t* __restrict__ src, int64_t K,
                                           int my_row, int nd, uint8_t* __restrict__ xq,
                                           float* __restrict__ sa, int64_t R, int lane) {
-    const int nseg = (int)((K + 255) / 256);
-    for (int s0 = 0; s0 < nseg; s0 += 4) {
-        uint4 v[4];
-        bool ok[4];
+    const int ntile = (int)(K / 128);
+    const int g = lane >> 3, j = lane & 7;
+    for (int t0 = 0; t0 < ntile; t0 += 8) {
+        uint4 v[2][2];
+        bool ok[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t off = (int64_t)(s0 + u) * 256 + 8 * lane;
-            ok[u] = (s0 + u < nseg) && (off < K);
-            v[u] = ok[u] ? fg8::ld_stream16(src + off) : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < 2; ++u) {
+            const int tile = t0 + 4 * u + g;
+            ok[u] = tile < ntile;
+            const uint16_t* p = src + (int64_t)tile * 128 + 8 * j;
+            v[u][0] = ok[u] ? fg8::ld_stream16(p) : make_uint4(0u, 0u, 0u, 0u);
+            v[u][1] = ok[u] ? fg8::ld_stream16(p + 64) : make_uint4(0u, 0u, 0u, 0u);
         }
-        // amax of the 4 tiles this half-warp holds (independent shuffle chains)
-        float m[4];
+        float m[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) m[u] = fg8::amax8(v[u]);
+        for (int u = 0; u < 2; ++u) m[u] = fmaxf(fg8::amax8(v[u][0]), fg8::amax8(v[u][1]));
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1)
+        for (int o = 4; o > 0; o >>= 1)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) m[u] = fmaxf(m[u], __shfl_xor_sync(kFull, m[u], o));
-        // fast-path codes of all 4 segments first, one combined check
-        float s[4];
-        fg8::QScale q[4];
-        uint2 c[4], h[4];
+            for (int u = 0; u < 2; ++u) m[u] = fmaxf(m[u], __shfl_xor_sync(kFull, m[u], o));
+        // fast-path codes of both groups first, one combined check
+        float s[2];
+        fg8::QScale q[2];
+        uint2 c[2][2], h[2][2];
         bool fast = true;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 2; ++u) {
             s[u] = fg8::tile_scale(m[u]);
             q[u] = fg8::make_qscale(s[u]);
-            fg8::quant8_bracket(v[u], q[u], c[u], h[u]);
-            fast &= !q[u].exact && fg8::bracket_agrees(c[u], h[u]);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                fg8::quant8_bracket(v[u][x], q[u], c[u][x], h[u][x]);
+                fast &= !q[u].exact && fg8::bracket_agrees(c[u][x], h[u][x]);
+            }
         }
         if (!fast) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (q[u].exact || !fg8::bracket_agrees(c[u], h[u])) c[u] = fg8::quant8_exact(v[u], q[u]);
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+                    if (q[u].exact || !fg8::bracket_agrees(c[u][x], h[u][x]))
+                        c[u][x] = fg8::quant8_exact(v[u][x], q[u]);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (s0 + u >= nseg) break;                 // warp-uniform
-            const int64_t off = (int64_t)(s0 + u) * 256 + 8 * lane;
-            const int64_t kb = (int64_t)(s0 + u) * 2 + (lane >> 4);
-            for (int j = 0; j < nd; ++j) {
-                const int r = __shfl_sync(kFull, my_row, j);
+        for (int u = 0; u < 2; ++u) {
+            const int tile = t0 + 4 * u + g;
+            const int64_t off = (int64_t)tile * 128 + 8 * j;
+            for (int d = 0; d < nd; ++d) {
+                const int r = __shfl_sync(kFull, my_row, d);
                 if (ok[u] && r >= 0) {
-                    *reinterpret_cast<uint2*>(xq + (int64_t)r * K + off) = c[u];
-                    if ((lane & 15) == 0) sa[kb * R + r] = s[u];
+                    uint8_t* dst = xq + (int64_t)r * K + off;
+                    *reinterpret_cast<uint2*>(dst) = c[u][0];
+                    *reinterpret_cast<uint2*>(dst + 64) = c[u][1];
+                    if (j == 0) sa[(int64_t)tile * R + r] = s[u];
                 }
             }
         }
