@@ -165,6 +165,28 @@ FG8_DEV void quant8xN(const uint4 (&v)[N], const QScale& q, uint2 (&c)[N]) {
     }
 }
 
+// Quantize 8 fp32 values (four pairs) with scale context q -> 8 codes.  Same
+// bracketed fast path as quant8, on fp32 inputs.
+FG8_DEV uint2 quant8f(float2 a, float2 b, float2 c, float2 d, const QScale& q) {
+    const float2 v[4] = {a, b, c, d};
+    const uint64_t rl = pack_f32x2(q.r_lo, q.r_lo), rh = pack_f32x2(q.r_hi, q.r_hi);
+    uint32_t l[4], h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t x = pack_f32x2(v[i].x, v[i].y);
+        l[i] = cvt_e4m3x2(mul_f32x2(x, rl));
+        h[i] = cvt_e4m3x2(mul_f32x2(x, rh));
+    }
+    uint2 lo = make_uint2(l[0] | (l[1] << 16), l[2] | (l[3] << 16));
+    const uint2 hi = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+    if (q.exact || !bracket_agrees(lo, hi)) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) l[i] = cvt_e4m3x2(__fdiv_rn(v[i].x, q.s), __fdiv_rn(v[i].y, q.s));
+        lo = make_uint2(l[0] | (l[1] << 16), l[2] | (l[3] << 16));
+    }
+    return lo;
+}
+
 // max |x| over 8 bf16 values: magnitudes of non-NaN floats order like their
 // bit patterns, so a 16-bit SIMD unsigned max over the sign-cleared words is exact.
 FG8_DEV float amax8(const uint4& v) {

@@ -125,7 +125,7 @@ struct Layout {
     static constexpr uint32_t kOffStages = 0;
     static constexpr uint32_t kOffBars = kStages * kStageBytes;
     // full, empty, tfull, tempty, drain (+ tile ring full / empty, contraction-grouped)
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kGroupK ? 2 * kTileRing : 0);
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kGroupK ? 2 * kTileRing : 2);
     static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;   // tmem slot, abort flag
     static constexpr uint32_t kOffRing = align_up(kOffMisc + 16, 16);  // int4 [kTileRing]
     // row-grouped: tiles per expert, exclusive prefix; contraction-grouped:
@@ -154,6 +154,11 @@ struct GemmArgs {
     void* out;
     int32_t* status;
     unsigned int* tile_ctr;   // contraction-grouped: zeroed tile counter
+    // row-grouped gate/up mode: B holds [gate; up] (N = 2 I rows per expert),
+    // out = E4M3 codes of h = silu(gate) * up [M_total][I], out_scale = their
+    // 1x128 scales [I/128][M_total]
+    int swiglu;
+    float* out_scale;
 };
 
 // ---------------------------------------------------------------------------
@@ -225,6 +230,19 @@ FG8_DEV void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// 64 fp32 values of this thread -> 32 lanes x 64 consecutive TMEM columns
+// (the 32x32b shape: a thread's values go to its own lane).  Completed by
+// tcgen05.wait::st.
+FG8_DEV void tmem_st64(uint32_t taddr, const float2* v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};\n"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0].x)), "r"(__float_as_uint(v[0].y)), "r"(__float_as_uint(v[1].x)), "r"(__float_as_uint(v[1].y)), "r"(__float_as_uint(v[2].x)), "r"(__float_as_uint(v[2].y)), "r"(__float_as_uint(v[3].x)), "r"(__float_as_uint(v[3].y)), "r"(__float_as_uint(v[4].x)), "r"(__float_as_uint(v[4].y)), "r"(__float_as_uint(v[5].x)), "r"(__float_as_uint(v[5].y)), "r"(__float_as_uint(v[6].x)), "r"(__float_as_uint(v[6].y)), "r"(__float_as_uint(v[7].x)), "r"(__float_as_uint(v[7].y)), "r"(__float_as_uint(v[8].x)), "r"(__float_as_uint(v[8].y)), "r"(__float_as_uint(v[9].x)), "r"(__float_as_uint(v[9].y)), "r"(__float_as_uint(v[10].x)), "r"(__float_as_uint(v[10].y)), "r"(__float_as_uint(v[11].x)), "r"(__float_as_uint(v[11].y)), "r"(__float_as_uint(v[12].x)), "r"(__float_as_uint(v[12].y)), "r"(__float_as_uint(v[13].x)), "r"(__float_as_uint(v[13].y)), "r"(__float_as_uint(v[14].x)), "r"(__float_as_uint(v[14].y)), "r"(__float_as_uint(v[15].x)), "r"(__float_as_uint(v[15].y)), "r"(__float_as_uint(v[16].x)), "r"(__float_as_uint(v[16].y)), "r"(__float_as_uint(v[17].x)), "r"(__float_as_uint(v[17].y)), "r"(__float_as_uint(v[18].x)), "r"(__float_as_uint(v[18].y)), "r"(__float_as_uint(v[19].x)), "r"(__float_as_uint(v[19].y)), "r"(__float_as_uint(v[20].x)), "r"(__float_as_uint(v[20].y)), "r"(__float_as_uint(v[21].x)), "r"(__float_as_uint(v[21].y)), "r"(__float_as_uint(v[22].x)), "r"(__float_as_uint(v[22].y)), "r"(__float_as_uint(v[23].x)), "r"(__float_as_uint(v[23].y)), "r"(__float_as_uint(v[24].x)), "r"(__float_as_uint(v[24].y)), "r"(__float_as_uint(v[25].x)), "r"(__float_as_uint(v[25].y)), "r"(__float_as_uint(v[26].x)), "r"(__float_as_uint(v[26].y)), "r"(__float_as_uint(v[27].x)), "r"(__float_as_uint(v[27].y)), "r"(__float_as_uint(v[28].x)), "r"(__float_as_uint(v[28].y)), "r"(__float_as_uint(v[29].x)), "r"(__float_as_uint(v[29].y)), "r"(__float_as_uint(v[30].x)), "r"(__float_as_uint(v[30].y)), "r"(__float_as_uint(v[31].x)), "r"(__float_as_uint(v[31].y))
+                 : "memory");
+}
+
+// silu(g) * u = g / (1 + e^-g) * u, fast exponential and division (the
+// result is quantized to E4M3 next; both are within a few fp32 ulps)
+FG8_DEV float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
 FG8_DEV uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -243,6 +261,7 @@ struct Tile {
     int nkb;            // 128-wide contraction blocks
     int64_t rowA;       // first operand-A row
     int64_t rowB;       // first operand-B row
+    int64_t rowB2;      // gate/up mode: first row of the up block (second half of B)
     int64_t out_row0;   // first output row
 };
 
@@ -265,7 +284,8 @@ FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const int32_t* s_off,
     T.e = lo;
     const int local = tile - s_tiles[lo];
     const int mt = local / nt, ntile = local - mt * nt;
-    T.n0 = ntile * BN;
+    // gate/up mode: a tile is 128 output columns, its B is gate block + up block
+    T.n0 = a.swiglu ? ntile * 128 : ntile * BN;
     const int32_t o0 = s_off[lo], o1 = s_off[lo + 1];
     T.rowA = (int64_t)o0 + (int64_t)mt * BM;
     // rows past M_total (offsets inconsistent with the buffers) are never touched
@@ -274,6 +294,7 @@ FG8_DEV Tile decode_tile(int tile, const int32_t* s_tiles, const int32_t* s_off,
     T.kx0 = 0;
     T.nkb = a.K / BK;
     T.rowB = (int64_t)lo * a.N + T.n0;
+    T.rowB2 = (int64_t)lo * a.N + a.N / 2 + T.n0;
     T.out_row0 = T.rowA;
     return T;
 }
@@ -298,6 +319,7 @@ FG8_DEV Tile decode_tile_k(int g, const int32_t* s_order, const int32_t* s_off, 
     T.kx0 = min(max(o0, 0), a.K) & ~(BK - 1);
     T.nkb = max(0, min(o1, a.K) - T.kx0) / BK;
     T.rowB = T.n0;
+    T.rowB2 = -1;
     T.out_row0 = (int64_t)e * a.M_total + T.rowA;
     return T;
 }
@@ -354,7 +376,7 @@ FG8_DEV bool ring_take(TileRing& R, bool whole_warp, int4& v, volatile int* abor
 // the kernel
 // ---------------------------------------------------------------------------
 
-template <bool kGroupK>
+template <bool kGroupK, bool kSwiglu = false>
 __global__ void __launch_bounds__(Warps<kGroupK>::kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
@@ -377,6 +399,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+    // row-grouped gate/up epilogue: one exchange barrier per TMEM buffer (a
+    // buffer is reused only after the gate warps have released it, so an
+    // exchange can never complete twice before the gate warps see it)
+    auto xchg_bar = [&](uint32_t b) { return bar0 + 8u * (2 * kStages + 5 + b); };
     const uint32_t ring_full0 = bar0 + 8u * (2 * kStages + 5);
     const uint32_t ring_empty0 = ring_full0 + 8u * kTileRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -386,7 +412,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     int32_t* s_warp = reinterpret_cast<int32_t*>(smem + kOffWarp);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nt = (a.N + BN - 1) / BN;
+    const int nt = (!kGroupK && kSwiglu) ? a.N / 256 : (a.N + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -398,6 +424,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             mbar_init(tempty_bar(b), kEpiWarps);
         }
         mbar_init(drain_bar, 1);
+        if (!kGroupK)
+            for (int b = 0; b < 2; ++b) mbar_init(xchg_bar(b), kEpiWarps / 2);
         if (kGroupK) {
             for (int i = 0; i < kTileRing; ++i) {
                 mbar_init(ring_full0 + 8u * i, 1);
@@ -494,7 +522,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
                     }
                     tma_load_2d(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA);
-                    tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
+                    if (!kGroupK && kSwiglu) {   // B map boxes are 128 rows here
+                        tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
+                        tma_load_2d(&tmB, sA + kABytes + kBBytes / 2, full_bar(stage), T.kx0 + kb * BK,
+                                    (int)T.rowB2);
+                    } else {
+                        tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
+                    }
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -574,6 +608,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int NB = a.N / 128, KBt = a.K / BK;
         uint32_t buf = 0, bphase = 0, sc = 0;
         uint32_t nbox = 0;    // TMA-store boxes issued by this warp (contraction-grouped)
+        uint32_t xphase = 0;  // gate/up epilogue: bit b = phase of xchg_bar(b)
         int e_hint = 0;
         bool ok = true;
         for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
@@ -613,8 +648,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 row_ok = r < T.rows_valid;
                 col0 = T.n0 + kCols * grp;
                 col_ok = col0 < a.N;
+                // gate/up mode: both halves cover output columns n0..n0+127; the
+                // second half's B rows (and block scales) are the up block
+                const int bcol = kSwiglu ? (grp == 0 ? T.n0 : a.N / 2 + T.n0) : col0;
+                if (kSwiglu) {
+                    col0 = T.n0;
+                    col_ok = true;
+                }
                 sa_p = a.sa + T.rowA + r;
-                sb_p = a.sb + ((int64_t)T.e * NB + col0 / 128) * KBt;
+                sb_p = a.sb + ((int64_t)T.e * NB + bcol / 128) * KBt;
             }
             // row-grouped mode: the scales of the next K block are loaded while
             // this one is promoted (two blocks ahead measured slower in the full
@@ -693,14 +735,91 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty_bar(buf));
+                // gate/up mode: the last K block's buffer carries the up values to
+                // the gate warps in the epilogue and is released there
+                if (kGroupK || !kSwiglu || kb + 1 < nkb) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty_bar(buf));
+                }
                 buf ^= 1u;
                 if (buf == 0) bphase ^= 1u;
             }
             if (!ok) break;
-            if (kGroupK) {
+            if (!kGroupK && kSwiglu) {
+                // Epilogue (gate/up): h = silu(gate) * up for this row's 128
+                // columns, quantized as one 1x128 tile.  The up warps park their
+                // accumulators in columns 128..255 of the last K block's TMEM
+                // buffer (same lanes), the gate warps read them back, form h and
+                // its codes and scale, and both release the buffer.
+                const uint32_t lbuf = buf ^ 1u;
+                const uint32_t xaddr = tmem_base + ((uint32_t)(32 * quarter) << 16) + lbuf * BN + 128;
+                if (grp == 1) {
+                    tmem_st64(xaddr, acc);
+                    tmem_st64(xaddr + 64, acc + 32);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(xchg_bar(lbuf));
+                } else {
+                    // bounded wait for the four up warps of this tile
+                    if (!mbar_wait(xchg_bar(lbuf), (xphase >> lbuf) & 1u, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    xphase ^= 1u << lbuf;
+                    tc_fence_after();
+                    float amax = 0.f;
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        uint32_t u[64];
+                        tmem_ld64(xaddr + 64 * ch, u);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            float2& g = acc[32 * ch + i];
+                            g.x = silu_mul(g.x, __uint_as_float(u[2 * i]));
+                            g.y = silu_mul(g.y, __uint_as_float(u[2 * i + 1]));
+                            amax = fmaxf(amax, fmaxf(fabsf(g.x), fabsf(g.y)));
+                        }
+                    }
+                    const float sc = fg8::tile_scale(amax);
+                    const fg8::QScale q = fg8::make_qscale(sc);
+                    // 128 codes of this thread's row, 16 at a time, through the
+                    // warp's staging rows: each store writes 8 rows x 64 bytes
+                    uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kOffStage) + ep * 32 * kStageWords;
+                    uint4* my_row = reinterpret_cast<uint4*>(stg + lane * kStageWords);
+                    const int sub = ((lane >> 2) & 1) * 4 + (lane >> 3);
+                    const int quad = lane & 3;
+                    uint8_t* ob = static_cast<uint8_t*>(a.out) + col0 + 16 * quad;
+                    const int I = a.N / 2;
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            uint2 c[2];
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const int base = 32 * ch + 8 * w4 + 4 * hh;   // float2 index: 8 values
+                                c[hh] = fg8::quant8f(acc[base], acc[base + 1], acc[base + 2], acc[base + 3], q);
+                            }
+                            my_row[w4] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int rr = 8 * g + sub;
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
+                            if (32 * quarter + rr < rows_valid)
+                                *reinterpret_cast<uint4*>(ob + (int64_t)(out_row0 + 32 * quarter + rr) * I + 64 * ch) = v;
+                        }
+                        __syncwarp();
+                    }
+                    if (row_ok) a.out_scale[(int64_t)(col0 / 128) * a.M_total + out_row0 + r] = sc;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(lbuf));
+            } else if (kGroupK) {
                 // Epilogue (contraction-grouped, fp32, full 128-row tiles): each
                 // warp writes its 32 rows x 128 columns as four 32 x 32 boxes,
                 // two at a time through its two 4 KB staging buffers, and
@@ -909,6 +1028,8 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     args.out = out;
     args.status = dev_status;
     args.tile_ctr = nullptr;
+    args.swiglu = 0;
+    args.out_scale = nullptr;
     if (group_mode == FG8_GROUP_K) {
         args.tile_ctr = take_tile_counter((cudaStream_t)stream);
         if (args.tile_ctr == nullptr) return FG8_ERR_CUDA;
@@ -917,5 +1038,58 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     if (grid > max_tiles) grid = max_tiles;
     if (grid < 1) grid = 1;
     kern<<<(unsigned)grid, threads, smem_bytes, (cudaStream_t)stream>>>(mA, mB, mOut, args);
+    return fg8h::launch_status();
+}
+
+extern "C" fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const float* sa,
+                                                    const uint8_t* b, const float* sb,
+                                                    const int32_t* offsets, int64_t M_total, int I,
+                                                    int K, int E, uint8_t* hq, float* sh,
+                                                    int32_t* dev_status, fg8_stream_t stream) {
+    if (!a || !sa || !b || !sb || !offsets || !hq || !sh) return FG8_ERR_INVALID_ARG;
+    if (E < 1 || I < 128 || K < 128 || I % 128 || K % 128 || M_total < 0)
+        return FG8_ERR_INVALID_ARG;
+    if (E > kMaxE) return FG8_ERR_UNSUPPORTED;
+    if (!fg8h::aligned16(a) || !fg8h::aligned16(b) || !fg8h::aligned16(hq) ||
+        (reinterpret_cast<uintptr_t>(sa) & 3) || (reinterpret_cast<uintptr_t>(sb) & 3) ||
+        (reinterpret_cast<uintptr_t>(sh) & 3) || (reinterpret_cast<uintptr_t>(offsets) & 3))
+        return FG8_ERR_INVALID_ARG;
+    if (M_total > INT32_MAX || (int64_t)E * 2 * I > INT32_MAX) return FG8_ERR_UNSUPPORTED;
+    if (M_total == 0) return FG8_OK;
+    const int64_t max_tiles = (M_total / BM + E) * (int64_t)(I / 128);
+    if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
+    CUtensorMap mA, mB;
+    // B boxes of 128 rows: a tile's gate block and up block land as the two
+    // halves of the 256-row operand tile
+    if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||
+        !make_map(&mB, b, (uint64_t)E * 2 * I, (uint64_t)K, 128))
+        return FG8_ERR_CUDA;
+    auto kern = grouped_gemm_kernel<false, true>;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, (const void*)kern) != cudaSuccess) return FG8_ERR_CUDA;
+    if (fa.numRegs < Warps<false>::kLaunchRegs) return FG8_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Layout<false>::kSmemBytes) != cudaSuccess)
+        return FG8_ERR_CUDA;
+    GemmArgs args;
+    args.sa = sa;
+    args.sb = sb;
+    args.offsets = offsets;
+    args.M_total = M_total;
+    args.N = 2 * I;
+    args.K = K;
+    args.E = E;
+    args.mode = FG8_GROUP_M;
+    args.out_f32 = 0;
+    args.out = hq;
+    args.status = dev_status;
+    args.tile_ctr = nullptr;
+    args.swiglu = 1;
+    args.out_scale = sh;
+    int64_t grid = fg8h::num_sms();
+    if (grid > max_tiles) grid = max_tiles;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, Warps<false>::kThreads, Layout<false>::kSmemBytes, (cudaStream_t)stream>>>(
+        mA, mB, mA, args);
     return fg8h::launch_status();
 }

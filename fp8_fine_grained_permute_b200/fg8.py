@@ -79,6 +79,9 @@ def lib() -> ctypes.CDLL:
         L.fg8_transpose_blockq.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P]
         L.fg8_grouped_gemm.restype = _I
         L.fg8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.fg8_grouped_gemm_swiglu_quant.restype = _I
+        L.fg8_grouped_gemm_swiglu_quant.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _P, _P,
+                                                    _P, _P]
         L.fg8_selftest_wait_timeout.restype = _I
         L.fg8_selftest_wait_timeout.argtypes = [_I, _P, _P, _P]
         L.fg8_status_string.restype = ctypes.c_char_p
@@ -175,6 +178,14 @@ def fg8_grouped_gemm(a, sa, b, sb, offsets, M_total, N, K, E, group_mode, bscale
                                   N, K, E, group_mode, bscale_mode, out_dtype, _ptr(out),
                                   _ptr(dev_status), _stream(stream)),
            "fg8_grouped_gemm")
+
+
+def fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, sh, dev_status,
+                                  stream=None):
+    _check(lib().fg8_grouped_gemm_swiglu_quant(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(offsets),
+                                               M_total, I, K, E, _ptr(hq), _ptr(sh),
+                                               _ptr(dev_status), _stream(stream)),
+           "fg8_grouped_gemm_swiglu_quant")
 
 
 def fg8_selftest_wait_timeout(which, scratch, dev_status, stream=None):
@@ -301,3 +312,19 @@ def grouped_gemm(a, sa, b, sb, offsets, out_dtype=FG8_OUT_BF16, group_mode=FG8_G
     fg8_grouped_gemm(a, sa, b, sb, offsets, M_total, N, K, E, group_mode, bmode, out_dtype, out,
                      dev_status, stream)
     return out
+
+
+def grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, dev_status=None, hq=None, sh=None,
+                              stream=None):
+    """a [M,K] E4M3, b [E,2I,K] E4M3 (gate rows then up rows) -> (hq [M,I]
+    E4M3, sh [I/128,M] fp32): the 1x128 quantization of silu(gate) * up."""
+    M_total, K = a.shape
+    E = offsets.numel() - 1
+    I = b.shape[1] // 2
+    if hq is None:
+        hq = torch.empty((M_total, I), dtype=torch.uint8, device=a.device)
+    if sh is None:
+        sh = torch.empty((I // 128, M_total), dtype=torch.float32, device=a.device)
+    fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, sh, dev_status,
+                                  stream)
+    return hq, sh

@@ -232,6 +232,39 @@ fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa,
                             int32_t* dev_status, fg8_stream_t stream);
 
 /*
+ * fg8_grouped_gemm_swiglu_quant -- the expert up-projection with its gated
+ * activation and the down-projection's 1x128 input quantization fused into
+ * the GEMM epilogue.  The pages combine FP8 GEMMs with separately written
+ * non-GEMM kernels ([K2] FP8 paragraph; [DS] sec. 2.2, FP8 mixed precision)
+ * and quantize every activation that enters an FP8 GEMM in 1x128 tiles; they
+ * do not name the expert's activation function.  Reading taken here: the
+ * gated SiLU of DeepSeek-style experts,
+ *   h[r][i] = silu(G[r][i]) * U[r][i],  silu(g) = g / (1 + exp(-g)),
+ * with G and U the fp32 accumulators of the row-grouped GEMM against the gate
+ * and up halves of b (promoted exactly as in fg8_grouped_gemm), and h
+ * quantized from fp32 (never rounded to bf16) as 1x128 tiles: for every row
+ * r and block c, sh[c][r] = amax/448 (1 for an all-zero tile) and
+ * hq[r][128c + j] = E4M3 RNE-satfinite(h / sh[c][r]).
+ *   a        E4M3 [M_total][K]; sa fp32 [K/128][M_total]
+ *   b        E4M3 [E][2I][K]: rows [0, I) of expert e are the gate weight,
+ *            rows [I, 2I) the up weight (fg8_quantize_weight of [E][2I][K])
+ *   sb       fp32 [E][2I/128][K/128]
+ *   offsets  int32 [E+1] on the device, as for FG8_GROUP_M
+ *   hq       E4M3 [M_total][I] and sh fp32 [I/128][M_total] (the layout
+ *            fg8_grouped_gemm takes as a and sa); rows outside
+ *            [0, offsets[E]) are not written
+ *   I % 128 == 0, K % 128 == 0, E <= 1024; a, b, hq 16-byte aligned.
+ * silu uses the fast exponential and division intrinsics (a few ulp in fp32).
+ * Errors as fg8_grouped_gemm; a timed-out internal wait writes
+ * FG8_ERR_TIMEOUT to *dev_status.
+ */
+fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const float* sa,
+                                         const uint8_t* b, const float* sb,
+                                         const int32_t* offsets, int64_t M_total, int I, int K,
+                                         int E, uint8_t* hq, float* sh, int32_t* dev_status,
+                                         fg8_stream_t stream);
+
+/*
  * fg8_selftest_wait_timeout -- diagnostic of the failure-detection path (the
  * pages have no counterpart).  Runs one of the library's bounded device waits
  * on a condition that nothing satisfies, so that it runs out after its limit

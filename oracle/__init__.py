@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
                                                  _P, _P, _I64, _P, _P]
         L.fg8o_gemm_kgrouped_entries.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I64, _I64,
                                                  _P, _P, _P, _I64, _P, _P]
+        L.fg8o_swiglu_quantize.argtypes = [_P, _P, _I64, _I64, _P, _P, _P]
     return _lib
 
 
@@ -230,6 +231,21 @@ def gemm_mgrouped_full(a, sa, b, sb, offsets):
     r, c = np.meshgrid(np.arange(M_total), np.arange(N), indexing="ij")
     ref, bound = gemm_mgrouped_entries(a, sa, b, sb, offsets, r.ravel(), c.ravel())
     return ref.reshape(M_total, N), bound.reshape(M_total, N)
+
+
+def swiglu_quantize(G, U):
+    """h = silu(G) * U in fp64, quantized in 1x128 tiles from its fp32 rounding.
+
+    G, U: fp64 [R, I].  Returns (h fp64 [R, I], hq u8 [R, I], sh f32 [I/128, R]).
+    """
+    G = np.ascontiguousarray(G, np.float64)
+    U = np.ascontiguousarray(U, np.float64)
+    R, I = G.shape
+    h = np.zeros((R, I), np.float64)
+    hq = np.zeros((R, I), np.uint8)
+    sh = np.zeros((I // 128, R), np.float32)
+    lib().fg8o_swiglu_quantize(_ptr(G), _ptr(U), R, I, _ptr(h), _ptr(hq), _ptr(sh))
+    return h, hq, sh
 
 
 def gemm_kgrouped_entries(a, sa, b, sb, padoff, experts, rows, cols):

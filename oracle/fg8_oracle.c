@@ -390,6 +390,47 @@ void fg8o_gemm_mgrouped_entries(const uint8_t* a, const float* sa, int64_t M_tot
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* gated activation of the up-projection, re-quantized in 1x128 tiles        */
+/* ------------------------------------------------------------------------ */
+
+/* The pages run most GEMMs in FP8 and quantize every activation that enters
+ * one in 1x128 tiles (Kanana-2 deep dive, FP8 paragraph; DeepSeek-V3 summary,
+ * sec. 2.2); they do not name the experts' activation.  Reading taken: the
+ * gated SiLU of DeepSeek-style experts,
+ *     h = silu(g) * u,   silu(g) = g / (1 + exp(-g)),
+ * evaluated in fp64 from the fp64 up-projection (g: gate half, u: up half),
+ * then rounded once to fp32 and quantized as 1x128 tiles exactly as above
+ * (amax of the fp32 values, s = fp32_RN(amax / 448), q = E4M3(fp32_RN(h / s))).
+ *   G, U  fp64 [R][I] (row-major), I % 128 == 0
+ *   h     fp64 [R][I] out: the activation before rounding (may be NULL)
+ *   hq    E4M3 [R][I];  sh fp32 [I/128][R]: sh[c*R + r] scales row r, block c */
+void fg8o_swiglu_quantize(const double* G, const double* U, int64_t R, int64_t I,
+                          double* h, uint8_t* hq, float* sh)
+{
+    float* hf = (float*)malloc(sizeof(float) * 128);
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t c = 0; c < I / 128; ++c) {
+            float amax = 0.0f;
+            for (int i = 0; i < 128; ++i) {
+                int64_t idx = r * I + c * 128 + i;
+                double g = G[idx];
+                double v = g / (1.0 + exp(-g)) * U[idx];
+                if (h)
+                    h[idx] = v;
+                hf[i] = (float)v;
+                if (fabsf(hf[i]) > amax)
+                    amax = fabsf(hf[i]);
+            }
+            float s = fg8o_tile_scale(amax);
+            for (int i = 0; i < 128; ++i)
+                hq[r * I + c * 128 + i] = quant_elem(hf[i], s);
+            sh[c * R + r] = s;
+        }
+    }
+    free(hf);
+}
+
 /* Contraction-grouped (weight gradient) product, one entry at a time:
  *   dW[e][m][n] = sum_{p in [padoff[e], padoff[e+1])}
  *                 dq(a[m][p]) * sa[p/128][m] * dq(b[n][p]) * sb[p/128][n]
