@@ -92,9 +92,12 @@ def padded_total_of(cfg: W.MoEConfig) -> int:
     return int(((counts + 127) // 128 * 128).sum())
 
 
-def work_of(cfg: W.MoEConfig, padded_total: int):
+def work_of(cfg: W.MoEConfig, padded_total: int, fused_act: bool = False):
     """Per kernel family of one step: (bound, algorithmic amount) and, for the
-    GEMMs, the bytes they must move at least (operands once, output once)."""
+    GEMMs, the bytes they must move at least (operands once, output once).
+    fused_act: the up-projection emits the quantized gated activation (E4M3
+    codes and 1x128 scales of H) instead of bf16 Y, and H is not quantized
+    separately."""
     T, K, k, E, R, N, I = cfg.T, cfg.hidden, cfg.k, cfg.E, cfg.R, cfg.n_up, cfg.inter
     w = {
         "quant_act_permute": ("hbm", bytes_route_quant(T, K, k, E)),
@@ -116,6 +119,11 @@ def work_of(cfg: W.MoEConfig, padded_total: int):
     if I:
         w["gemm_fprop_down"] = ("tensor", 2 * R * K * I)
         gemm_bytes["gemm_fprop_down"] = R * I + E * K * I + 2 * R * K
+    if fused_act and I:
+        del w["gemm_fprop_up"], gemm_bytes["gemm_fprop_up"]
+        w["gemm_fprop_up_swiglu_quant"] = ("tensor", 2 * R * N * K)
+        gemm_bytes["gemm_fprop_up_swiglu_quant"] = R * K + E * N * K + R * I + 4 * R * (I // 128)
+        w["quant_act_rows"] = ("hbm", bytes_rows_quant(R, N))
     return w, gemm_bytes
 
 
@@ -180,11 +188,12 @@ def measured_traffic(family: str, cfg: W.MoEConfig, padded_total: int):
 class Step:
     """Device-resident inputs and outputs of one step; `run` launches the path."""
 
-    def __init__(self, cfg: W.MoEConfig, dev):
+    def __init__(self, cfg: W.MoEConfig, dev, fused_act: bool = False):
         from fp8_fine_grained_permute_b200 import fg8
         self.fg8 = fg8
         self.cfg = cfg
         self.dev = dev
+        self.fused_act = bool(fused_act and cfg.inter)
         T, K, k, E, R = cfg.T, cfg.hidden, cfg.k, cfg.E, cfg.R
         N, I = cfg.n_up, cfg.inter
         self.ids_np = W.route(cfg)
@@ -197,7 +206,7 @@ class Step:
         self.ids = torch.from_numpy(self.ids_np).to(dev)
         self.w_up = W.gen_w_up(cfg, dev)
         self.w_down = W.gen_w_down(cfg, dev) if I else None
-        self.h = W.gen_h(cfg, dev) if I else None
+        self.h = W.gen_h(cfg, dev) if I and not self.fused_act else None
         self.dy = W.gen_dy(cfg, dev)
         # outputs / intermediates
         self.xq, self.sa = e((R, K), u8), e((K // 128, R), f32)
@@ -207,7 +216,7 @@ class Step:
         self.ws = e(self.ws_bytes, u8)
         self.status = torch.zeros(1, dtype=i32, device=dev)
         self.wq_up, self.sw_up = e((E, N, K), u8), e((E, N // 128, K // 128), f32)
-        self.y_up = e((R, N), bf)
+        self.y_up = e((R, N), bf) if not self.fused_act else None
         if I:
             self.wq_dn, self.sw_dn = e((E, K, I), u8), e((E, K // 128, I // 128), f32)
             self.hq, self.sh = e((R, I), u8), e((I // 128, R), f32)
@@ -220,7 +229,7 @@ class Step:
         self.xT, self.sxT, self.pad_x = e((K, self.P), u8), e((self.P // 128, K), f32), e(E + 1, i32)
         self.dw = e((E, N, K), f32)
         self.launches_per_step = 0
-        self.work, self.gemm_bytes = work_of(cfg, self.padded_total)
+        self.work, self.gemm_bytes = work_of(cfg, self.padded_total, self.fused_act)
 
     def run(self, stream, marks=None):
         """Launch one step on `stream`.  With `marks`, record an event pair
@@ -260,12 +269,15 @@ class Step:
                 fg8.fg8_quantize_weight(u16(self.w_down), E, K, I, self.wq_dn, self.sw_dn, self.status, sp)
                 n[0] += 1
         timed("quant_weight", wquant)
-        timed("gemm_fprop_up", launch(lambda: fg8.fg8_grouped_gemm(
-            self.xq, self.sa, self.wq_up, self.sw_up, self.offsets, R, N, K, E, fg8.FG8_GROUP_M,
-            fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_up, self.status, sp)))
+        if self.fused_act:
+            timed("gemm_fprop_up_swiglu_quant", launch(lambda: self.run_fused_up(stream)))
+        else:
+            timed("gemm_fprop_up", launch(lambda: fg8.fg8_grouped_gemm(
+                self.xq, self.sa, self.wq_up, self.sw_up, self.offsets, R, N, K, E, fg8.FG8_GROUP_M,
+                fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_up, self.status, sp)))
 
         def rows():
-            if I:
+            if I and not self.fused_act:
                 fg8.fg8_quantize_act(u16(self.h), R, I, None, 1, 1, None, fg8.FG8_ROWWISE, self.hq,
                                      self.sh, None, None, None, None, None, None, 0, None, sp)
                 n[0] += 1
@@ -296,6 +308,14 @@ class Step:
             fg8.FG8_BSCALE_ROW128, fg8.FG8_OUT_F32, self.dw, self.status, sp)))
         self.launches_per_step = n[0]
 
+    def run_fused_up(self, stream):
+        """Up-projection with the gated activation and its 1x128 quantization
+        in the epilogue: X_q W_up -> (H_q, s_H), the down-projection's input."""
+        c = self.cfg
+        self.fg8.fg8_grouped_gemm_swiglu_quant(self.xq, self.sa, self.wq_up, self.sw_up,
+                                               self.offsets, c.R, c.inter, c.hidden, c.E,
+                                               self.hq, self.sh, self.status, stream.cuda_stream)
+
     def run_transpose(self, stream):
         """The standalone block transpose (fg8_transpose_blockq) of the up
         weight: the step gets WqT from the fused quantizer, this times the
@@ -310,7 +330,7 @@ class Step:
     IN_NAMES = ("x", "ids", "dy", "h")
 
     def out_names(self):
-        return ("y_dn" if self.h is not None else "y_up", "dx")
+        return ("y_dn" if self.cfg.inter else "y_up", "dx")
 
     def make_slots(self):
         names = [n for n in self.IN_NAMES if getattr(self, n) is not None] + list(self.out_names())
@@ -494,6 +514,10 @@ def main():
     ap.add_argument("--config", default="dsv3", choices=sorted(W.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fused-act", action="store_true",
+                    help="forward through the up-projection with the gated activation and its "
+                         "1x128 quantization fused in the epilogue (H comes from the up-projection "
+                         "instead of being a separate input)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -522,7 +546,7 @@ def main():
     fg8.lib()
 
     cfg = W.CONFIGS[args.config]
-    st = Step(cfg, dev)
+    st = Step(cfg, dev, fused_act=args.fused_act)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -601,6 +625,27 @@ def main():
                     "frac": tr_gb / pk["hbm_gbs"], "share": None,
                     "traffic": measured_traffic("transpose_blockq", cfg, st.padded_total),
                     "note": "not in the step: the step's WqT comes from the fused quantizer"})
+    # the fused up-projection + gated activation + 1x128 quantization on its own
+    # (outside the default step, which keeps the unfused chain)
+    if cfg.inter and not st.fused_act:
+        with torch.cuda.stream(stream):
+            st.run_fused_up(stream)
+            fu0, fu1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fu0.record(stream)
+            for _ in range(args.steps):
+                st.run_fused_up(stream)
+            fu1.record(stream)
+        torch.cuda.synchronize()
+        fu_ms = fu0.elapsed_time(fu1) / args.steps
+        fu_tf = 2.0 * cfg.R * cfg.n_up * cfg.hidden / (fu_ms * 1e-3) / 1e12
+        kernels.append({"kernel": "gemm_fprop_up_swiglu_quant", "standalone": True,
+                        "bound": "tensor", "ms": fu_ms, "achieved": fu_tf, "peak": fp8_peak,
+                        "unit": "TFLOP/s", "frac": fu_tf / fp8_peak, "share": None,
+                        "traffic": None,
+                        "replaces_ms": kern_ms["gemm_fprop_up"],
+                        "note": "not in the step: replaces gemm_fprop_up (bf16 Y) and the row "
+                                "quantization of H; back-to-back launches, operands L2-warm "
+                                "only in part (W_up alone exceeds L2)"})
     # whole job: every rank did the same work; divide by the slowest rank's time
     gemm_ms, q_ms = all_max(pg, [gemm_ms, q_ms], dev)
     gemm_tflops = job_rate(world, gemm_flops, gemm_ms) / 1e12
@@ -659,7 +704,7 @@ def main():
         e2e = {"value": job_rate(world, gemm_flops, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "GEMM FLOPs per step over the whole step time including pinned-host "
-                       "copies of X, ids, H, dY in and the forward output and dX out; two "
+                       f"copies of {', '.join(host_in)} in and {', '.join(host_out)} out; two "
                        "device slots, copies overlap the next step's kernels"}
     if st.status.item() != 0:
         raise RuntimeError(f"device status {fg8.status_name(st.status.item())}")
@@ -681,6 +726,7 @@ def main():
                        "E": cfg.E, "T": cfg.T, "k": cfg.k, "hidden": cfg.hidden,
                        "n_up": cfg.n_up, "inter": cfg.inter, "routed_rows": cfg.R,
                        "parallelism": f"replicas x{world}",
+                       "fused_act": st.fused_act,
                        "l2": "inputs larger than L2 (step working set > 50 GB)"},
             "quantize_gbs": quant_gbs,
             "gemm_frac_of_fp8_peak": gemm_tflops / world / fp8_peak,
