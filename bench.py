@@ -87,6 +87,12 @@ def bytes_transpose(E, N, K):
     return 2 * (E * N * K + 4 * E * N * K // 16384)
 
 
+def bytes_combine(T, k, C):
+    """Unpermute + combine: the k routed bf16 rows of every token in, its bf16
+    row out, plus the row index and affinity of every slot."""
+    return T * k * C * 2 + T * C * 2 + T * k * 8
+
+
 def padded_total_of(cfg: W.MoEConfig) -> int:
     counts = np.bincount(W.route(cfg).ravel(), minlength=cfg.E)
     return int(((counts + 127) // 128 * 128).sum())
@@ -315,6 +321,17 @@ class Step:
         self.fg8.fg8_grouped_gemm_swiglu_quant(self.xq, self.sa, self.wq_up, self.sw_up,
                                                self.offsets, c.R, c.inter, c.hidden, c.E,
                                                self.hq, self.sh, self.status, stream.cuda_stream)
+
+    def run_combine(self, stream):
+        """Unpermute + combine of the down-projection output: each token's k
+        rows summed with its normalized gate weights -> [T, hidden] bf16."""
+        c = self.cfg
+        if not hasattr(self, "comb_out"):
+            self.affinity = W.gen_affinity(c, self.dev)
+            self.comb_out = torch.empty((c.T, c.hidden), dtype=torch.bfloat16, device=self.dev)
+        self.fg8.fg8_unpermute_combine(self.y_dn.view(torch.int16), c.R, c.hidden, self.token_row,
+                                       self.affinity, c.T, c.k, 1, self.fg8.FG8_OUT_BF16,
+                                       self.comb_out, stream.cuda_stream)
 
     def run_transpose(self, stream):
         """The standalone block transpose (fg8_transpose_blockq) of the up
@@ -646,6 +663,25 @@ def main():
                         "note": "not in the step: replaces gemm_fprop_up (bf16 Y) and the row "
                                 "quantization of H; back-to-back launches, operands L2-warm "
                                 "only in part (W_up alone exceeds L2)"})
+    # unpermute + combine of the down-projection output on its own
+    if cfg.inter:
+        with torch.cuda.stream(stream):
+            st.run_combine(stream)
+            cb0, cb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            cb0.record(stream)
+            for _ in range(args.steps):
+                st.run_combine(stream)
+            cb1.record(stream)
+        torch.cuda.synchronize()
+        cb_ms = cb0.elapsed_time(cb1) / args.steps
+        cb_bytes = bytes_combine(cfg.T, cfg.k, cfg.hidden)
+        cb_gb = cb_bytes / (cb_ms * 1e-3) / 1e9
+        kernels.append({"kernel": "unpermute_combine", "standalone": True, "bound": "hbm",
+                        "ms": cb_ms, "achieved": cb_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": cb_gb / pk["hbm_gbs"], "share": None, "traffic": None,
+                        "note": "not in the step: the layer output after the down-projection "
+                                "(T x hidden bf16 from R routed rows); back-to-back launches, "
+                                "rows larger than L2"})
     # whole job: every rank did the same work; divide by the slowest rank's time
     gemm_ms, q_ms = all_max(pg, [gemm_ms, q_ms], dev)
     gemm_tflops = job_rate(world, gemm_flops, gemm_ms) / 1e12

@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.fg8_grouped_gemm_swiglu_quant.restype = _I
         L.fg8_grouped_gemm_swiglu_quant.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _P, _P,
                                                     _P, _P]
+        L.fg8_unpermute_combine.restype = _I
+        L.fg8_unpermute_combine.argtypes = [_P, _I64, _I, _P, _P, _I64, _I, _I, _I, _P, _P]
         L.fg8_selftest_wait_timeout.restype = _I
         L.fg8_selftest_wait_timeout.argtypes = [_I, _P, _P, _P]
         L.fg8_status_string.restype = ctypes.c_char_p
@@ -186,6 +188,13 @@ def fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, s
                                                M_total, I, K, E, _ptr(hq), _ptr(sh),
                                                _ptr(dev_status), _stream(stream)),
            "fg8_grouped_gemm_swiglu_quant")
+
+
+def fg8_unpermute_combine(y, R, C, token_row, affinity, T, k, normalize, out_dtype, out,
+                          stream=None):
+    _check(lib().fg8_unpermute_combine(_ptr(y), R, C, _ptr(token_row), _ptr(affinity), T, k,
+                                       normalize, out_dtype, _ptr(out), _stream(stream)),
+           "fg8_unpermute_combine")
 
 
 def fg8_selftest_wait_timeout(which, scratch, dev_status, stream=None):
@@ -328,3 +337,18 @@ def grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, dev_status=None, hq=None, s
     fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, sh, dev_status,
                                   stream)
     return hq, sh
+
+
+def unpermute_combine(y, token_row, affinity, normalize=True, out_dtype=FG8_OUT_BF16, out=None,
+                      stream=None):
+    """y bf16 [R, C] (permuted rows), token_row int32 [T*k], affinity fp32 [T, k]
+    -> out [T, C]: each token's rows summed with its (normalized) gate weights."""
+    R, C = y.shape
+    T, k = affinity.shape
+    if out is None:
+        dt = torch.float32 if out_dtype == FG8_OUT_F32 else torch.bfloat16
+        out = torch.empty((T, C), dtype=dt, device=affinity.device)
+    yv = y.view(torch.int16) if y.dtype == torch.bfloat16 else y
+    fg8_unpermute_combine(yv, R, C, token_row, affinity, T, k, int(bool(normalize)), out_dtype,
+                          out, stream)
+    return out

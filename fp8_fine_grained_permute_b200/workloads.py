@@ -261,6 +261,7 @@ CONFIGS = {
 
 # stream ids of the tensors of one configuration
 SID_X, SID_W_UP, SID_W_DOWN, SID_H, SID_DY = 1, 2, 3, 4, 5
+SID_Y_DOWN, SID_AFF = 6, 7
 SIGMA_X, SIGMA_W = 1.0, 0.02
 
 
@@ -310,6 +311,24 @@ def gen_dy(cfg: MoEConfig, device="cpu", row0: int = 0, rows: int | None = None)
     rows = cfg.R - row0 if rows is None else rows
     return gen_grad_bf16((rows, cfg.n_up), cfg.seed, SID_DY, device,
                          index_offset=row0 * cfg.n_up)
+
+
+def gen_y_down(cfg: MoEConfig, device="cpu") -> torch.Tensor:
+    """Down-projection output [R, hidden] in expert order (N(0, 1) bf16)."""
+    return gen_normal_bf16((cfg.R, cfg.hidden), 1.0, cfg.seed, SID_Y_DOWN, device)
+
+
+def gen_affinity(cfg: MoEConfig, device="cpu") -> torch.Tensor:
+    """Sigmoid affinities of each token's chosen experts [T, k], fp32 in (0, 1)."""
+    return gen_uniform_f32((cfg.T, cfg.k), cfg.seed, SID_AFF, device)
+
+
+def gen_uniform_f32(shape, seed: int, sid: int, device="cpu", index_offset: int = 0) -> torch.Tensor:
+    """fp32 values uniform on the 2^24-point grid (i + 0.5) / 2^24 of (0, 1)."""
+    numel = math.prod(shape)
+    idx = torch.arange(index_offset, index_offset + numel, dtype=torch.int64, device=device)
+    u = (hash_index(idx, seed, sid) >> 8).to(torch.float64)
+    return ((u + 0.5) / float(1 << 24)).to(torch.float32).view(*shape)
 
 
 # --------------------------------------------------------------------------

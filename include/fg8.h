@@ -265,6 +265,31 @@ fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const float* sa,
                                          fg8_stream_t stream);
 
 /*
+ * fg8_unpermute_combine -- the layer output of routed tokens: every token's
+ * expert output rows (one per routed slot, in the permuted expert order that
+ * fg8_quantize_act produced) summed with the gate weights ([DS] sec. 2.1:
+ * sigmoid affinity scores, top-K experts per token, no token dropping).  The
+ * page does not spell out how the affinities of the chosen experts become
+ * weights; reading taken here: they are normalized to sum 1 over the token's
+ * kept slots (normalize = 1), or used as given (normalize = 0).
+ *   out[t][c] = sum_{j < k, slot kept} w[t][j] * y[token_row[t*k + j]][c]
+ *   w[t][j]   = normalize ? affinity[t][j] / (sum of the kept affinity[t][.])
+ *                         : affinity[t][j]
+ * A slot is kept when token_row[t*k + j] is in [0, R); others (-1 = no row)
+ * add nothing.  Arithmetic in fp32 with every operation rounded to nearest
+ * (the affinity sum and the weighted sum in slot order j = 0, 1, ...); a
+ * normalized token whose kept affinities sum to 0 gets zeros.
+ *   y          bf16 [R][C] (e.g. the down-projection output), R may be 0
+ *   token_row  int32 [T*k] (fg8_quantize_act's token_row)
+ *   affinity   fp32 [T][k]
+ *   out        [T][C], bf16 (RNE of the fp32 sum) or fp32 (out_dtype)
+ *   1 <= k <= 16, C % 8 == 0; y and out 16-byte aligned.
+ */
+fg8_status fg8_unpermute_combine(const uint16_t* y, int64_t R, int C, const int32_t* token_row,
+                                 const float* affinity, int64_t T, int k, int normalize,
+                                 int out_dtype, void* out, fg8_stream_t stream);
+
+/*
  * fg8_selftest_wait_timeout -- diagnostic of the failure-detection path (the
  * pages have no counterpart).  Runs one of the library's bounded device waits
  * on a condition that nothing satisfies, so that it runs out after its limit

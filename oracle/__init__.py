@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.fg8o_gemm_kgrouped_entries.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I64, _I64,
                                                  _P, _P, _P, _I64, _P, _P]
         L.fg8o_swiglu_quantize.argtypes = [_P, _P, _I64, _I64, _P, _P, _P]
+        L.fg8o_unpermute_combine.argtypes = [_P, _I64, _I64, _P, _P, _I64, _I, _I, _P, _P]
     return _lib
 
 
@@ -246,6 +247,24 @@ def swiglu_quantize(G, U):
     sh = np.zeros((I // 128, R), np.float32)
     lib().fg8o_swiglu_quantize(_ptr(G), _ptr(U), R, I, _ptr(h), _ptr(hq), _ptr(sh))
     return h, hq, sh
+
+
+def unpermute_combine(y, token_row, affinity, normalize=True):
+    """fp64 layer output of routed tokens and the |term| sum of every entry.
+
+    y: bf16 [R, C] (uint16 bits or torch bf16); token_row int32 [T*k];
+    affinity fp32 [T, k].  Returns (out fp64 [T, C], bound fp64 [T, C]).
+    """
+    yu = _u16(y)
+    R, C = yu.shape
+    affinity = np.ascontiguousarray(affinity, np.float32)
+    token_row = np.ascontiguousarray(token_row, np.int32)
+    T, k = affinity.shape
+    out = np.zeros((T, C), np.float64)
+    bound = np.zeros((T, C), np.float64)
+    lib().fg8o_unpermute_combine(_ptr(yu), R, C, _ptr(token_row), _ptr(affinity), T, k,
+                                 int(bool(normalize)), _ptr(out), _ptr(bound))
+    return out, bound
 
 
 def gemm_kgrouped_entries(a, sa, b, sb, padoff, experts, rows, cols):

@@ -431,6 +431,49 @@ void fg8o_swiglu_quantize(const double* G, const double* U, int64_t R, int64_t I
     free(hf);
 }
 
+/* ------------------------------------------------------------------------ */
+/* unpermute + combine                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Each token's output is the sum of its routed slots' expert rows weighted by
+ * the gate values (DeepSeek-V3 summary, sec. 2.1: sigmoid affinities, top-K
+ * experts per token).  Reading taken: the gate values are the affinities of
+ * the token's kept slots normalized to sum 1 (normalize != 0), or the
+ * affinities as given.  A slot is kept when its row is in [0, R).  In fp64:
+ *   out[t][c]   = sum_j w[t][j] * y[token_row[t*k + j]][c]
+ *   bound[t][c] = sum_j |w[t][j] * y[...][c]|
+ *   y bf16 [R][C]; token_row int32 [T*k]; affinity fp32 [T][k]; out, bound fp64 [T][C].
+ * A normalized token whose kept affinities sum to 0 gets zeros. */
+void fg8o_unpermute_combine(const uint16_t* y, int64_t R, int64_t C, const int32_t* token_row,
+                            const float* affinity, int64_t T, int k, int normalize,
+                            double* out, double* bound)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        double sum = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int32_t row = token_row[t * k + j];
+            if (row >= 0 && row < R)
+                sum += (double)affinity[t * k + j];
+        }
+        for (int64_t c = 0; c < C; ++c) {
+            double acc = 0.0, mag = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int32_t row = token_row[t * k + j];
+                if (row < 0 || row >= R)
+                    continue;
+                double w = (double)affinity[t * k + j];
+                if (normalize)
+                    w = sum != 0.0 ? w / sum : 0.0;
+                double term = w * (double)fg8o_bf16_to_f32(y[(int64_t)row * C + c]);
+                acc += term;
+                mag += fabs(term);
+            }
+            out[t * C + c] = acc;
+            bound[t * C + c] = mag;
+        }
+    }
+}
+
 /* Contraction-grouped (weight gradient) product, one entry at a time:
  *   dW[e][m][n] = sum_{p in [padoff[e], padoff[e+1])}
  *                 dq(a[m][p]) * sa[p/128][m] * dq(b[n][p]) * sb[p/128][n]
