@@ -322,6 +322,18 @@ class Step:
                                                self.offsets, c.R, c.inter, c.hidden, c.E,
                                                self.hq, self.sh, self.status, stream.cuda_stream)
 
+    def run_route(self, stream):
+        """Sigmoid-affinity top-k routing of the step's tokens (ids and
+        affinities for the permuting quantizer and the combine)."""
+        c = self.cfg
+        if not hasattr(self, "logits"):
+            self.logits = W.gen_router_logits(c, self.dev)
+            self.rbias = W.gen_expert_bias(c, self.dev)
+            self.r_ids = torch.empty((c.T, c.k), dtype=torch.int32, device=self.dev)
+            self.r_aff = torch.empty((c.T, c.k), dtype=torch.float32, device=self.dev)
+        self.fg8.fg8_route_topk(self.logits, self.rbias, c.T, c.E, c.k, self.r_ids, self.r_aff,
+                                stream.cuda_stream)
+
     def run_combine(self, stream):
         """Unpermute + combine of the down-projection output: each token's k
         rows summed with its normalized gate weights -> [T, hidden] bf16."""
@@ -682,6 +694,23 @@ def main():
                         "note": "not in the step: the layer output after the down-projection "
                                 "(T x hidden bf16 from R routed rows); back-to-back launches, "
                                 "rows larger than L2"})
+    # sigmoid-affinity top-k routing on its own
+    with torch.cuda.stream(stream):
+        st.run_route(stream)
+        ro0, ro1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ro0.record(stream)
+        for _ in range(args.steps):
+            st.run_route(stream)
+        ro1.record(stream)
+    torch.cuda.synchronize()
+    ro_ms = ro0.elapsed_time(ro1) / args.steps
+    ro_gb = (cfg.T * cfg.E * 4 + cfg.E * 4 + cfg.T * cfg.k * 8) / (ro_ms * 1e-3) / 1e9
+    kernels.append({"kernel": "route_topk", "standalone": True, "bound": "hbm", "ms": ro_ms,
+                    "achieved": ro_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": ro_gb / pk["hbm_gbs"], "share": None, "traffic": None,
+                    "note": "not in the step (its ids come from the seeded host routing): "
+                            "T x E fp32 logits -> top-k ids and affinities; a few MB, "
+                            "L2-resident between launches, so launch- and latency-bound"})
     # whole job: every rank did the same work; divide by the slowest rank's time
     gemm_ms, q_ms = all_max(pg, [gemm_ms, q_ms], dev)
     gemm_tflops = job_rate(world, gemm_flops, gemm_ms) / 1e12

@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.fg8_grouped_gemm_swiglu_quant.restype = _I
         L.fg8_grouped_gemm_swiglu_quant.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _P, _P,
                                                     _P, _P]
+        L.fg8_route_topk.restype = _I
+        L.fg8_route_topk.argtypes = [_P, _P, _I64, _I, _I, _P, _P, _P]
         L.fg8_unpermute_combine.restype = _I
         L.fg8_unpermute_combine.argtypes = [_P, _I64, _I, _P, _P, _I64, _I, _I, _I, _P, _P]
         L.fg8_selftest_wait_timeout.restype = _I
@@ -188,6 +190,12 @@ def fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, s
                                                M_total, I, K, E, _ptr(hq), _ptr(sh),
                                                _ptr(dev_status), _stream(stream)),
            "fg8_grouped_gemm_swiglu_quant")
+
+
+def fg8_route_topk(logits, bias, T, E, k, ids, affinity, stream=None):
+    _check(lib().fg8_route_topk(_ptr(logits), _ptr(bias), T, E, k, _ptr(ids), _ptr(affinity),
+                                _stream(stream)),
+           "fg8_route_topk")
 
 
 def fg8_unpermute_combine(y, R, C, token_row, affinity, T, k, normalize, out_dtype, out,
@@ -352,3 +360,14 @@ def unpermute_combine(y, token_row, affinity, normalize=True, out_dtype=FG8_OUT_
     fg8_unpermute_combine(yv, R, C, token_row, affinity, T, k, int(bool(normalize)), out_dtype,
                           out, stream)
     return out
+
+
+def route_topk(logits, bias, k, ids=None, affinity=None, stream=None):
+    """logits fp32 [T, E], bias fp32 [E] -> (ids int32 [T, k], affinity fp32 [T, k])."""
+    T, E = logits.shape
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if affinity is None:
+        affinity = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    fg8_route_topk(logits, bias, T, E, k, ids, affinity, stream)
+    return ids, affinity

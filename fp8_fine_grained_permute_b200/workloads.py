@@ -261,7 +261,7 @@ CONFIGS = {
 
 # stream ids of the tensors of one configuration
 SID_X, SID_W_UP, SID_W_DOWN, SID_H, SID_DY = 1, 2, 3, 4, 5
-SID_Y_DOWN, SID_AFF = 6, 7
+SID_Y_DOWN, SID_AFF, SID_LOGITS, SID_BIAS = 6, 7, 8, 9
 SIGMA_X, SIGMA_W = 1.0, 0.02
 
 
@@ -321,6 +321,16 @@ def gen_y_down(cfg: MoEConfig, device="cpu") -> torch.Tensor:
 def gen_affinity(cfg: MoEConfig, device="cpu") -> torch.Tensor:
     """Sigmoid affinities of each token's chosen experts [T, k], fp32 in (0, 1)."""
     return gen_uniform_f32((cfg.T, cfg.k), cfg.seed, SID_AFF, device)
+
+
+def gen_router_logits(cfg: MoEConfig, device="cpu") -> torch.Tensor:
+    """Router logits [T, E] fp32 (N(0, 1) values on the bf16 grid)."""
+    return gen_normal_bf16((cfg.T, cfg.E), 1.0, cfg.seed, SID_LOGITS, device).to(torch.float32)
+
+
+def gen_expert_bias(cfg: MoEConfig, device="cpu") -> torch.Tensor:
+    """Per-expert routing bias [E] fp32, uniform on (-0.1, 0.1)."""
+    return (gen_uniform_f32((cfg.E,), cfg.seed, SID_BIAS, device) - 0.5) * 0.2
 
 
 def gen_uniform_f32(shape, seed: int, sid: int, device="cpu", index_offset: int = 0) -> torch.Tensor:

@@ -265,6 +265,23 @@ fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const float* sa,
                                          fg8_stream_t stream);
 
 /*
+ * fg8_route_topk -- sigmoid-affinity top-K routing with a per-expert bias
+ * ([DS] sec. 2.1: sigmoid affinity scores, top-K experts per token, a
+ * per-expert bias term adjusted for load balance instead of an auxiliary
+ * loss).  Reading taken here: the bias enters only the choice, the gate
+ * values use the plain affinities.  For every token t and expert e, in fp32:
+ *   s[e] = 1 / (1 + exp(-logits[t][e]))   (IEEE add and divide, accurate exp)
+ *   c[e] = s[e] + bias[e]
+ * ids[t][0..k) are the k experts with the largest c, in descending c, ties
+ * to the lower expert index; affinity[t][j] = s[ids[t][j]].  The outputs feed
+ * fg8_quantize_act (ids) and fg8_unpermute_combine (affinity).
+ *   logits fp32 [T][E]; bias fp32 [E]; ids int32 [T][k]; affinity fp32 [T][k]
+ *   1 <= k <= min(16, E), E <= 1024.  NaN logits are outside the contract.
+ */
+fg8_status fg8_route_topk(const float* logits, const float* bias, int64_t T, int E, int k,
+                          int32_t* ids, float* affinity, fg8_stream_t stream);
+
+/*
  * fg8_unpermute_combine -- the layer output of routed tokens: every token's
  * expert output rows (one per routed slot, in the permuted expert order that
  * fg8_quantize_act produced) summed with the gate weights ([DS] sec. 2.1:

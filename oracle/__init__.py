@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
                                                  _P, _P, _P, _I64, _P, _P]
         L.fg8o_swiglu_quantize.argtypes = [_P, _P, _I64, _I64, _P, _P, _P]
         L.fg8o_unpermute_combine.argtypes = [_P, _I64, _I64, _P, _P, _I64, _I, _I, _P, _P]
+        L.fg8o_route_topk.argtypes = [_P, _P, _I64, _I, _I, _P, _P, _P]
     return _lib
 
 
@@ -247,6 +248,22 @@ def swiglu_quantize(G, U):
     sh = np.zeros((I // 128, R), np.float32)
     lib().fg8o_swiglu_quantize(_ptr(G), _ptr(U), R, I, _ptr(h), _ptr(hq), _ptr(sh))
     return h, hq, sh
+
+
+def route_topk(logits, bias, k):
+    """Sigmoid-affinity top-k with a per-expert bias, in fp64.
+
+    logits fp32 [T, E], bias fp32 [E].  Returns (ids int32 [T, k],
+    affinity fp64 [T, k], score fp64 [T, E] = sigmoid(logits) + bias).
+    """
+    logits = np.ascontiguousarray(logits, np.float32)
+    bias = np.ascontiguousarray(bias, np.float32)
+    T, E = logits.shape
+    ids = np.zeros((T, k), np.int32)
+    aff = np.zeros((T, k), np.float64)
+    score = np.zeros((T, E), np.float64)
+    lib().fg8o_route_topk(_ptr(logits), _ptr(bias), T, E, k, _ptr(ids), _ptr(aff), _ptr(score))
+    return ids, aff, score
 
 
 def unpermute_combine(y, token_row, affinity, normalize=True):

@@ -432,6 +432,46 @@ void fg8o_swiglu_quantize(const double* G, const double* U, int64_t R, int64_t I
 }
 
 /* ------------------------------------------------------------------------ */
+/* sigmoid-affinity top-K routing with a per-expert bias                    */
+/* ------------------------------------------------------------------------ */
+
+/* DeepSeek-V3 summary, sec. 2.1: sigmoid affinity scores, the top-K experts
+ * per token, a per-expert bias adjusted for load balance.  Reading taken: the
+ * bias only ranks (c = s + b), the affinities written out are s.  In fp64:
+ *   s[e] = 1 / (1 + exp(-u[t][e])),  c[e] = s[e] + bias[e]
+ * K rounds, each taking the remaining expert with the largest c, ties to the
+ * lower index.  ids int32 [T][k]; affinity fp64 [T][k]; score fp64 [T][E]
+ * (c of every expert, may be NULL). */
+void fg8o_route_topk(const float* logits, const float* bias, int64_t T, int E, int k,
+                     int32_t* ids, double* affinity, double* score)
+{
+    double* s = (double*)malloc(sizeof(double) * (size_t)E);
+    double* c = (double*)malloc(sizeof(double) * (size_t)E);
+    char* taken = (char*)malloc((size_t)E);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            s[e] = 1.0 / (1.0 + exp(-(double)logits[t * E + e]));
+            c[e] = s[e] + (double)bias[e];
+            taken[e] = 0;
+            if (score)
+                score[t * E + e] = c[e];
+        }
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || c[e] > c[best]))
+                    best = e;              /* strict '>' keeps the lower index on ties */
+            taken[best] = 1;
+            ids[t * k + j] = best;
+            affinity[t * k + j] = s[best];
+        }
+    }
+    free(s);
+    free(c);
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------ */
 /* unpermute + combine                                                      */
 /* ------------------------------------------------------------------------ */
 

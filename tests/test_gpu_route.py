@@ -1,0 +1,111 @@
+"""GPU parity of the sigmoid-affinity top-K routing kernel against the oracle.
+
+The choice is an integer decision taken from fp32 scores on the GPU (accurate
+expf, IEEE add and divide) and fp64 scores in the oracle, so near-ties may
+resolve differently.  Checked: every row holds k distinct experts; the chosen
+set is a valid top-k of the fp64 scores up to eps = 2^-20 (well above the
+fp32 score error, a few ulps of values below 2) and in descending order up to
+eps; at least 99% of the rows equal the oracle's exactly; where scores tie
+exactly (integer logits) the lower index wins, bit for bit; the affinities are
+the sigmoid of the chosen logits within 2^-21 relative.
+"""
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+from fp8_fine_grained_permute_b200 import build as fbuild
+from fp8_fine_grained_permute_b200 import fg8
+
+pytestmark = pytest.mark.gpu
+
+EPS = 2.0 ** -20
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    fbuild.build()
+    fg8.lib()
+    torch.cuda.init()
+
+
+def run(u, b, k):
+    ids, aff = fg8.route_topk(torch.from_numpy(u).cuda(), torch.from_numpy(b).cuda(), k)
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), aff.cpu().numpy()
+
+
+def check(oracle, u, b, k, exact_frac=0.99, what=""):
+    T, E = u.shape
+    ids, aff = run(u, b, k)
+    ids_o, _, score = oracle.route_topk(u, b, k)
+    assert ids.min() >= 0 and ids.max() < E, what
+    srt = np.sort(ids, axis=1)
+    assert np.all(np.diff(srt, axis=1) > 0), f"{what}: repeated expert"
+    c = np.take_along_axis(score, ids.astype(np.int64), 1)
+    mask = np.ones((T, E), bool)
+    np.put_along_axis(mask, ids.astype(np.int64), False, 1)
+    rest = np.where(mask, score, -np.inf).max(axis=1) if k < E else np.full(T, -np.inf)
+    assert np.all(c.min(axis=1) >= rest - EPS), f"{what}: not a top-{k}"
+    assert np.all(np.diff(c, axis=1) <= EPS), f"{what}: not in descending order"
+    same = np.all(ids == ids_o, axis=1)
+    assert np.mean(same) >= exact_frac, f"{what}: {np.mean(~same)} rows differ"
+    s = expit(np.take_along_axis(u, ids.astype(np.int64), 1).astype(np.float64))
+    assert np.all(np.abs(aff - s) <= 2.0 ** -21 * s + 1e-38), f"{what}: affinity"
+
+
+@pytest.mark.parametrize("T,E,k", [(1000, 64, 6), (700, 256, 8), (300, 33, 4), (50, 7, 7),
+                                   (200, 1000, 16), (64, 1, 1), (129, 512, 2)])
+def test_route_matches_oracle(oracle, T, E, k):
+    rng = np.random.default_rng(T * 7 + E * 3 + k)
+    u = rng.standard_normal((T, E)).astype(np.float32)
+    b = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    check(oracle, u, b, k, what=f"T={T} E={E} k={k}")
+
+
+def test_route_exact_ties_lower_index(oracle):
+    rng = np.random.default_rng(91)
+    T, E, k = 500, 96, 8
+    u = rng.integers(-1, 2, (T, E)).astype(np.float32)
+    b = np.zeros(E, np.float32)
+    ids, _ = run(u, b, k)
+    ids_o, _, _ = oracle.route_topk(u, b, k)
+    np.testing.assert_array_equal(ids, ids_o)
+
+
+def test_route_dsv3_size(oracle):
+    rng = np.random.default_rng(92)
+    T, E, k = 8192, 256, 8
+    u = rng.standard_normal((T, E)).astype(np.float32)
+    b = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    check(oracle, u, b, k, what="dsv3")
+
+
+def test_route_feeds_the_permuting_quantizer(oracle):
+    """The ids go straight into fg8_quantize_act: its expert offsets must be
+    the histogram of the chosen ids (no bad id)."""
+    rng = np.random.default_rng(93)
+    T, E, k, K = 640, 32, 4, 256
+    u = torch.from_numpy(rng.standard_normal((T, E)).astype(np.float32)).cuda()
+    b = torch.from_numpy(rng.uniform(-0.1, 0.1, E).astype(np.float32)).cuda()
+    ids, _ = fg8.route_topk(u, b, k)
+    x = torch.randn((T, K), generator=torch.Generator().manual_seed(94)).to(torch.bfloat16).cuda()
+    st = fg8.new_status()
+    out = fg8.quantize_act(x, ids, E, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    counts = np.bincount(ids.cpu().numpy().ravel(), minlength=E)
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(),
+                                  np.concatenate([[0], np.cumsum(counts)]))
+
+
+def test_route_rejects_bad_arguments():
+    u = torch.zeros((4, 8), device="cuda")
+    b = torch.zeros(8, device="cuda")
+    ids = torch.empty((4, 17), dtype=torch.int32, device="cuda")
+    aff = torch.empty((4, 17), device="cuda")
+    for E, k in [(8, 9), (8, 17), (2000, 4), (8, 0)]:
+        with pytest.raises(fg8.FG8Error) as ei:
+            fg8.fg8_route_topk(u, b, 4, E, k, ids, aff)
+        assert ei.value.status == fg8.FG8_ERR_INVALID_ARG
