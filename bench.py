@@ -142,26 +142,33 @@ def work_of(cfg: W.MoEConfig, padded_total: int, fused_act: bool = False):
 TRAFFIC_CAPTURE = {
     "config": "kanana",
     "families": {
-        "quant_act_permute": (224.8e6, "quant_act", "20970841eab1"),
-        "quant_weight": (1026.8e6, "quant_weight", "9614c0fc5313"),
-        "gemm_fprop_up": (680.9e6, "gemm", "c4c6456bac63"),
-        "gemm_fprop_down": (530.8e6, "gemm", "c4c6456bac63"),
-        "transpose_blockq": (345.9e6, "transpose", "c1e4961cfa8c"),
-        "quant_act_rows": (627.0e6, "quant_act", "20970841eab1"),
-        "gemm_dgrad": (722.5e6, "gemm", "c4c6456bac63"),
-        "quant_act_colwise": (664.7e6, "quant_act", "20970841eab1"),
-        "gemm_wgrad": (1151.7e6, "gemm", "c4c6456bac63"),
+        "quant_act_permute": (225.1e6, "quant_act", "2c6776891a41"),
+        "quant_weight": (1023.6e6, "quant_weight", "3fdb1d33d509"),
+        "gemm_fprop_up": (680.3e6, "gemm", "0263c351d655"),
+        "gemm_fprop_down": (530.7e6, "gemm", "0263c351d655"),
+        "transpose_blockq": (345.9e6, "transpose", "5fbbb56efbb6"),
+        "quant_act_rows": (624.1e6, "quant_act", "2c6776891a41"),
+        "gemm_dgrad": (722.0e6, "gemm", "0263c351d655"),
+        "quant_act_colwise": (663.7e6, "quant_act", "2c6776891a41"),
+        "gemm_wgrad": (1151.4e6, "gemm", "0263c351d655"),
+        "gemm_fprop_up_swiglu_quant": (479.1e6, "gemm", "0263c351d655"),
+        "unpermute_combine": (446.9e6, "combine", "e28e1d5711ca"),
     },
 }
+# the files each family's counters depend on; fg8_common.cuh is added unless
+# the group lists its own headers (the transpose uses none of its device code
+# but one unchanged load helper)
 _SRC = {"quant_act": ["quant_act.cu", "fg8_tma.cuh"], "quant_weight": ["quant_weight.cu", "fg8_tma.cuh"],
-        "transpose": ["transpose_blockq.cu"], "gemm": ["grouped_gemm.cu", "fg8_tma.cuh"]}
+        "transpose": ["transpose_blockq.cu"], "gemm": ["grouped_gemm.cu", "fg8_tma.cuh"],
+        "combine": ["combine.cu"]}
+_OWN_HEADERS = {"transpose"}
 
 
 def source_hash(group: str) -> str:
     import hashlib
     h = hashlib.sha1()
     base = os.path.join(ROOT, "fp8_fine_grained_permute_b200", "csrc")
-    for f in _SRC[group] + ["fg8_common.cuh"]:
+    for f in _SRC[group] + ([] if group in _OWN_HEADERS else ["fg8_common.cuh"]):
         with open(os.path.join(base, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
@@ -171,6 +178,11 @@ def algorithmic_bytes(family: str, cfg: W.MoEConfig, padded_total: int) -> float
     """The bytes a family must move on `cfg` (GEMMs: operands + output once)."""
     if family == "transpose_blockq":
         return bytes_transpose(cfg.E, cfg.n_up, cfg.hidden)
+    if family == "unpermute_combine":
+        return bytes_combine(cfg.T, cfg.k, cfg.hidden)
+    if family == "gemm_fprop_up_swiglu_quant":
+        R, K, I = cfg.R, cfg.hidden, cfg.inter
+        return R * K + cfg.E * cfg.n_up * K + R * I + 4 * R * (I // 128)
     w, gb = work_of(cfg, padded_total)
     return gb.get(family, w[family][1])
 
@@ -670,7 +682,7 @@ def main():
         kernels.append({"kernel": "gemm_fprop_up_swiglu_quant", "standalone": True,
                         "bound": "tensor", "ms": fu_ms, "achieved": fu_tf, "peak": fp8_peak,
                         "unit": "TFLOP/s", "frac": fu_tf / fp8_peak, "share": None,
-                        "traffic": None,
+                        "traffic": measured_traffic("gemm_fprop_up_swiglu_quant", cfg, st.padded_total),
                         "replaces_ms": kern_ms["gemm_fprop_up"],
                         "note": "not in the step: replaces gemm_fprop_up (bf16 Y) and the row "
                                 "quantization of H; back-to-back launches, operands L2-warm "
@@ -690,7 +702,8 @@ def main():
         cb_gb = cb_bytes / (cb_ms * 1e-3) / 1e9
         kernels.append({"kernel": "unpermute_combine", "standalone": True, "bound": "hbm",
                         "ms": cb_ms, "achieved": cb_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": cb_gb / pk["hbm_gbs"], "share": None, "traffic": None,
+                        "frac": cb_gb / pk["hbm_gbs"], "share": None,
+                        "traffic": measured_traffic("unpermute_combine", cfg, st.padded_total),
                         "note": "not in the step: the layer output after the down-projection "
                                 "(T x hidden bf16 from R routed rows); back-to-back launches, "
                                 "rows larger than L2"})
