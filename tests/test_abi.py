@@ -74,6 +74,40 @@ def test_null_and_shape_arguments_rejected_on_host(L):
                               16, 1 << 20, None, None) == fg8.FG8_ERR_UNSUPPORTED  # k > 32
 
 
+def test_next_entry_points_reject_bad_arguments_on_host(L):
+    INV, OK = fg8.FG8_ERR_INVALID_ARG, fg8.FG8_OK
+    F32 = fg8.FG8_OUT_F32
+    # gated-activation up-projection: I % 128, K % 128, null outputs, misaligned codes
+    assert L.fg8_grouped_gemm_swiglu_quant(16, 16, 16, 16, 16, 128, 96, 128, 1, 16, 16, None,
+                                           None) == INV
+    assert L.fg8_grouped_gemm_swiglu_quant(16, 16, 16, 16, 16, 128, 128, 100, 1, 16, 16, None,
+                                           None) == INV
+    assert L.fg8_grouped_gemm_swiglu_quant(16, 16, 16, 16, 16, 128, 128, 128, 1, None, 16, None,
+                                           None) == INV
+    assert L.fg8_grouped_gemm_swiglu_quant(16, 16, 16, 16, 16, 128, 128, 128, 1, 24, 16, None,
+                                           None) == INV
+    assert L.fg8_grouped_gemm_swiglu_quant(16, 16, 16, 16, 16, 128, 128, 128, 2000, 16, 16, None,
+                                           None) == fg8.FG8_ERR_UNSUPPORTED       # E > 1024
+    assert L.fg8_grouped_gemm_swiglu_quant(16, 16, 16, 16, 16, 0, 128, 128, 1, 16, 16, None,
+                                           None) == OK                            # no rows
+    # combine: slots, row width, flags, dtype; an empty batch is a no-op
+    assert L.fg8_unpermute_combine(16, 8, 16, 16, 16, 4, 17, 1, F32, 16, None) == INV
+    assert L.fg8_unpermute_combine(16, 8, 12, 16, 16, 4, 2, 1, F32, 16, None) == INV
+    assert L.fg8_unpermute_combine(16, 8, 16, 16, 16, 4, 2, 2, F32, 16, None) == INV
+    assert L.fg8_unpermute_combine(16, 8, 16, 16, 16, 4, 2, 1, 5, 16, None) == INV
+    assert L.fg8_unpermute_combine(16, 8, 16, None, 16, 4, 2, 1, F32, 16, None) == INV
+    assert L.fg8_unpermute_combine(16, 8, 16, 16, 16, 4, 2, 1, F32, 24, None) == INV   # out align
+    assert L.fg8_unpermute_combine(None, 0, 16, None, None, 0, 2, 1, F32, None, None) == OK
+    # routing: k within [1, min(16, E)], E <= 1024; an empty batch is a no-op
+    assert L.fg8_route_topk(16, 16, 4, 8, 9, 16, 16, None) == INV
+    assert L.fg8_route_topk(16, 16, 4, 64, 17, 16, 16, None) == INV
+    assert L.fg8_route_topk(16, 16, 4, 2000, 4, 16, 16, None) == INV
+    assert L.fg8_route_topk(16, 16, 4, 64, 0, 16, 16, None) == INV
+    assert L.fg8_route_topk(None, 16, 4, 64, 4, 16, 16, None) == INV
+    assert L.fg8_route_topk(18, 16, 4, 64, 4, 16, 16, None) == INV                     # align
+    assert L.fg8_route_topk(None, None, 0, 64, 4, None, None, None) == OK
+
+
 def test_binding_refuses_cpu_tensors(L):
     import torch
     w = torch.zeros((1, 128, 128), dtype=torch.bfloat16)
