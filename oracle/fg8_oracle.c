@@ -22,6 +22,13 @@
  *    bullets.
  *  - GEMM partial sums are promoted to high precision (fp32 on the GPU); the
  *    oracle sums in fp64: DeepSeek-V3 summary, sec. 2.2, third bullet.
+ *  - Around the expert GEMMs (each with the reading it takes stated where it
+ *    is defined below): sigmoid-affinity top-K routing with a per-expert bias
+ *    and the weighted combine of a token's expert outputs (DeepSeek-V3
+ *    summary, sec. 2.1), and the gated activation between the two expert
+ *    GEMMs, re-quantized in 1x128 tiles for the second (Kanana-2 deep dive,
+ *    FP8 paragraph; DeepSeek-V3 summary, sec. 2.2).  These are computed in
+ *    fp64 throughout.
  *
  * The pages fix neither the FP8 format nor the scale formula.  This oracle
  * takes one reading and states it: OCP "E4M3FN" (bias 7, no infinities, NaN =
