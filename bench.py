@@ -138,21 +138,22 @@ def work_of(cfg: W.MoEConfig, padded_total: int, fused_act: bool = False):
 # the DeepSeek-V3-shaped step is too large to capture under full sets).  They
 # are scaled to another workload by the ratio of algorithmic bytes, and
 # dropped (traffic: null) when the kernel sources differ from the ones the
-# counters were taken on (short sha1 of the kernel file + shared headers).
+# counters were taken on (short sha1 of the code of the kernel file and shared
+# headers, comments and whitespace removed).
 TRAFFIC_CAPTURE = {
     "config": "kanana",
     "families": {
-        "quant_act_permute": (225.1e6, "quant_act", "2c6776891a41"),
-        "quant_weight": (1023.6e6, "quant_weight", "3fdb1d33d509"),
-        "gemm_fprop_up": (680.3e6, "gemm", "0263c351d655"),
-        "gemm_fprop_down": (530.7e6, "gemm", "0263c351d655"),
-        "transpose_blockq": (345.9e6, "transpose", "5fbbb56efbb6"),
-        "quant_act_rows": (624.1e6, "quant_act", "2c6776891a41"),
-        "gemm_dgrad": (722.0e6, "gemm", "0263c351d655"),
-        "quant_act_colwise": (663.7e6, "quant_act", "2c6776891a41"),
-        "gemm_wgrad": (1151.4e6, "gemm", "0263c351d655"),
-        "gemm_fprop_up_swiglu_quant": (479.1e6, "gemm", "0263c351d655"),
-        "unpermute_combine": (446.9e6, "combine", "e28e1d5711ca"),
+        "quant_act_permute": (225.1e6, "quant_act", "3d397202c14b"),
+        "quant_weight": (1023.6e6, "quant_weight", "6dd6a32fa993"),
+        "gemm_fprop_up": (680.3e6, "gemm", "5e2d6565d807"),
+        "gemm_fprop_down": (530.7e6, "gemm", "5e2d6565d807"),
+        "transpose_blockq": (345.9e6, "transpose", "3f2c2c5f91b7"),
+        "quant_act_rows": (624.1e6, "quant_act", "3d397202c14b"),
+        "gemm_dgrad": (722.0e6, "gemm", "5e2d6565d807"),
+        "quant_act_colwise": (663.7e6, "quant_act", "3d397202c14b"),
+        "gemm_wgrad": (1151.4e6, "gemm", "5e2d6565d807"),
+        "gemm_fprop_up_swiglu_quant": (479.1e6, "gemm", "5e2d6565d807"),
+        "unpermute_combine": (446.9e6, "combine", "08a271eae050"),
     },
 }
 # the files each family's counters depend on; fg8_common.cuh is added unless
@@ -164,13 +165,39 @@ _SRC = {"quant_act": ["quant_act.cu", "fg8_tma.cuh"], "quant_weight": ["quant_we
 _OWN_HEADERS = {"transpose"}
 
 
+def code_of(text: str) -> str:
+    """C/CUDA source without comments and blank space (what the counters
+    depend on): string literals are kept, // and /* */ comments dropped, runs
+    of whitespace folded."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def source_hash(group: str) -> str:
     import hashlib
     h = hashlib.sha1()
     base = os.path.join(ROOT, "fp8_fine_grained_permute_b200", "csrc")
     for f in _SRC[group] + ([] if group in _OWN_HEADERS else ["fg8_common.cuh"]):
-        with open(os.path.join(base, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(base, f), encoding="utf-8") as fh:
+            h.update(code_of(fh.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -36,6 +36,13 @@
 // (row-grouped mode); in the contraction-grouped mode an expert with no tokens
 // writes zeros.
 //
+// Gate/up mode (row-grouped, fg8_grouped_gemm_swiglu_quant): a tile is 128
+// rows x 128 output columns whose 256-row B operand is the expert's gate block
+// and up block for those columns (two 128-row TMA boxes), so warpgroup 0
+// accumulates the gate and warpgroup 1 the up projection; after the last K
+// block the up values are handed to the gate warps through TMEM and the
+// epilogue writes silu(gate) * up as E4M3 codes with one scale per 1x128 tile.
+//
 // Every mbarrier wait is bounded (FG8_ERR_TIMEOUT in *status, then the roles
 // wind down and TMEM is released); the kernel never traps.
 #include <cuda.h>
@@ -49,9 +56,11 @@ namespace {
 
 using namespace fg8::tma;
 
-// 128 x 256 tiles: N = 256 is the widest single-CTA tcgen05.mma, and narrower
-// ones do not pay (128 x 128 tiles with four TMEM buffers were measured at
-// 0.6x the throughput: an N = 128 MMA takes nearly as long as an N = 256 one).
+// 128 x 256 tiles: N = 256 is the widest single-CTA tcgen05.mma.  Narrower
+// tiles do not pay here: 128 x 128 tiles with four TMEM buffers ran at 0.6x the
+// throughput, because the promotion's fixed cost per K block (waits, fences,
+// buffer release, scale loads) is then spread over half the work, although an
+// N = 128 MMA on its own takes half the time of an N = 256 one.
 constexpr int BM = 128, BN = 256, BK = 128;
 constexpr uint32_t kABytes = BM * BK;              // 16 KB
 constexpr uint32_t kBBytes = BN * BK;              // 32 KB
