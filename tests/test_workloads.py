@@ -56,3 +56,24 @@ def test_routing_structure():
         assert np.array_equal(ids, W.route(cfg))             # deterministic
     counts = np.bincount(W.route(W.CONFIGS["dsv3"]).ravel(), minlength=256)
     assert (counts == 0).sum() == 16 and counts.max() > 4000  # Zipf skew + forced empties
+
+
+def test_routing_kernel_and_combine_inputs():
+    cfg = W.CONFIGS["tiny"]
+    aff = W.gen_affinity(cfg)
+    assert aff.shape == (cfg.T, cfg.k) and aff.dtype == torch.float32
+    assert float(aff.min()) > 0.0 and float(aff.max()) < 1.0
+    assert torch.equal(aff, W.gen_affinity(cfg))
+    # the 2^24-point grid: every value is (i + 0.5) / 2^24 rounded to fp32
+    u = W.gen_uniform_f32((1000,), 7, 3)
+    i = torch.floor(u.double() * 2 ** 24)
+    assert torch.all(((i + 0.5) / 2 ** 24).float() == u)
+    assert torch.equal(W.gen_uniform_f32((10,), 7, 3, index_offset=990), u[990:])
+    logits = W.gen_router_logits(cfg)
+    assert logits.shape == (cfg.T, cfg.E) and logits.dtype == torch.float32
+    assert torch.equal(logits.to(torch.bfloat16).float(), logits)      # bf16-grid values
+    b = W.gen_expert_bias(cfg)
+    assert b.shape == (cfg.E,) and float(b.abs().max()) < 0.1
+    y = W.gen_y_down(cfg)
+    assert y.shape == (cfg.R, cfg.hidden) and y.dtype == torch.bfloat16
+    assert abs(float(y.float().std()) - 1.0) < 0.1
