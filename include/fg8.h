@@ -25,7 +25,10 @@
  *  - All data pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, never synchronizes the stream and keeps no state
  *    between calls, so calls on different streams with disjoint buffers are
- *    independent.  `stream` is a cudaStream_t (NULL = the legacy stream).
+ *    independent, with two stated exceptions: the contraction-grouped GEMM's
+ *    tile counters (fg8_grouped_gemm) and the allocation-free quantizer's
+ *    scratch (fg8_quantize_act_noalloc) are device memory of the library.
+ *    `stream` is a cudaStream_t (NULL = the legacy stream).
  *  - bf16 data is passed as uint16_t bit patterns.  FP8 data as uint8_t.
  *  - Calls are asynchronous.  Argument errors are found on the host and
  *    returned immediately (nothing is launched).  Launch failures return
