@@ -273,6 +273,7 @@ class Step:
         self.dyT, self.sdyT, self.pad_dy = e((N, self.P), u8), e((self.P // 128, N), f32), e(E + 1, i32)
         self.xT, self.sxT, self.pad_x = e((K, self.P), u8), e((self.P // 128, K), f32), e(E + 1, i32)
         self.dw = e((E, N, K), f32)
+        self.gemm_ws = e(max(16, fg8.fg8_grouped_gemm_workspace(fg8.FG8_GROUP_K)), u8)
         self.launches_per_step = 0
         self.work, self.gemm_bytes = work_of(cfg, self.padded_total, self.fused_act)
 
@@ -319,7 +320,7 @@ class Step:
         else:
             timed("gemm_fprop_up", launch(lambda: fg8.fg8_grouped_gemm(
                 self.xq, self.sa, self.wq_up, self.sw_up, self.offsets, R, N, K, E, fg8.FG8_GROUP_M,
-                fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_up, self.status, sp)))
+                fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_up, None, 0, self.status, sp)))
 
         def rows():
             if I and not self.fused_act:
@@ -334,10 +335,10 @@ class Step:
             timed("gemm_fprop_down", launch(lambda: fg8.fg8_grouped_gemm(
                 self.hq, self.sh, self.wq_dn, self.sw_dn, self.offsets, R, K, I, E,
                 fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.y_dn,
-                self.status, sp)))
+                None, 0, self.status, sp)))
         timed("gemm_dgrad", launch(lambda: fg8.fg8_grouped_gemm(
             self.dyq, self.sdy, self.wqT_up, self.swT_up, self.offsets, R, K, N, E,
-            fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.dx, self.status, sp)))
+            fg8.FG8_GROUP_M, fg8.FG8_BSCALE_BLOCK128, fg8.FG8_OUT_BF16, self.dx, None, 0, self.status, sp)))
 
         def colwise():
             fg8.fg8_quantize_act(u16(self.dy), R, N, None, 1, E, self.offsets, fg8.FG8_COLWISE,
@@ -350,8 +351,23 @@ class Step:
         timed("quant_act_colwise", colwise)
         timed("gemm_wgrad", launch(lambda: fg8.fg8_grouped_gemm(
             self.dyT, self.sdyT, self.xT, self.sxT, self.pad_dy, N, K, self.P, E, fg8.FG8_GROUP_K,
-            fg8.FG8_BSCALE_ROW128, fg8.FG8_OUT_F32, self.dw, self.status, sp)))
+            fg8.FG8_BSCALE_ROW128, fg8.FG8_OUT_F32, self.dw, self.gemm_ws, self.gemm_ws.numel(),
+            self.status, sp)))
         self.launches_per_step = n[0]
+
+    def run_up_alternative(self, stream):
+        """The up-projection variant the step does not run (for a standalone
+        timing on the same operands)."""
+        c = self.cfg
+        if self.fused_act:
+            if not hasattr(self, "y_up_alt"):
+                self.y_up_alt = torch.empty((c.R, c.n_up), dtype=torch.bfloat16, device=self.dev)
+            self.fg8.fg8_grouped_gemm(self.xq, self.sa, self.wq_up, self.sw_up, self.offsets, c.R,
+                                      c.n_up, c.hidden, c.E, self.fg8.FG8_GROUP_M,
+                                      self.fg8.FG8_BSCALE_BLOCK128, self.fg8.FG8_OUT_BF16,
+                                      self.y_up_alt, None, 0, self.status, stream.cuda_stream)
+        else:
+            self.run_fused_up(stream)
 
     def run_fused_up(self, stream):
         """Up-projection with the gated activation and its 1x128 quantization
@@ -470,52 +486,242 @@ class ClockSampler:
 # CPU oracle timing (cpu_baseline and the reference arm)
 # --------------------------------------------------------------------------
 
-class OracleSample:
-    """The oracle, as it stands, on a bounded sample of the workload: permute +
-    1x128 quantize of the first tokens, 128x128 quantize and transpose of a
-    slab of one expert's up-projection weight, and the fp64 GEMM of whole
-    output rows against that expert.  Inputs are generated once, outside the
-    timed calls."""
+class OracleBaseline:
+    """The oracle, as it stands (never tuned for timing), on this host's cores,
+    on the workload of the step: K1 (permute + 1x128 quantize of X, identity-
+    mode rows of dY, column-wise dY and gathered X), K2 (both weights), K3 (the
+    up weight) and the fp64 GEMM.  Rates use the algorithmic byte and FLOP
+    formulas of the GPU line, so the numbers compare.
 
-    def __init__(self, cfg: W.MoEConfig, ntok: int = 32, wrows: int = 512):
+    The work is cut into units the method never couples (token slabs, row
+    slabs, experts or 128-row slabs of an expert's weight, output rows); each
+    unit is one call of the oracle's plain single-threaded function.
+    `time_1t` runs a few units of every family on one thread; `time_all` runs
+    each family over a pool of threads, one unit per thread at a time: over
+    the whole configuration when the per-family time budget allows, else over
+    the first units that fit (reported as the fraction `covered`).  The GEMM
+    at full size would take hours in fp64 on the host: it is timed on sampled
+    output rows and its full-size time extrapolated (labelled so).
+
+    Inputs are the seeded generators' output, untimed: copied from the device
+    tensors of the GPU step (`source`, whole experts), or generated on the
+    host (`source` None: 128-row weight slabs and smaller activation slabs,
+    prepared once and reused, for the reference arm's bounded steps)."""
+
+    FAMILIES = ("quant_act_permute", "quant_act_rows", "quant_act_colwise", "quant_weight",
+                "transpose_blockq")
+
+    def __init__(self, cfg: W.MoEConfig, source=None):
         import oracle
         oracle.build()
         self.o = oracle
         self.cfg = cfg
-        K, N, E = cfg.hidden, cfg.n_up, cfg.E
-        ids = W.route(cfg)
-        counts = np.bincount(ids.ravel(), minlength=E)
-        self.e = int(np.argmax(counts))
-        self.ntok = ntok
-        self.ids = np.ascontiguousarray(ids[:ntok])
-        self.x = W.gen_x(cfg)[:ntok].contiguous()
-        self.wrows = min(wrows, N)
-        self.w = W.gen_w_up(cfg, experts=[self.e])[:, :self.wrows].contiguous()
-        act = oracle.quantize_act(self.x[:8].contiguous(), None, 1)
-        self.a_rows, self.sa_rows = act["xq"], act["sa"]
-        self.q_bytes = (bytes_route_quant(ntok, K, cfg.k, E) + bytes_weight_quant(1, self.wrows, K) +
-                        bytes_transpose(1, self.wrows, K))
+        self.src = source
+        self.small = source is None
+        self.ids = W.route(cfg)
+        self.route = oracle.route(self.ids, cfg.E)
+        self.counts = np.diff(self.route["offsets"])
+        self.nz = [int(e) for e in np.nonzero(self.counts)[0]]
+        self._x = None
 
-    def run(self, gemm_budget_s: float):
-        o, K = self.o, self.cfg.hidden
-        t0 = time.perf_counter()
-        o.quantize_act(self.x, self.ids, self.cfg.E)
-        wq, sw = o.quantize_weight(self.w)
-        o.transpose_blockq(wq, sw)
-        t_quant = time.perf_counter() - t0
-        rows, flops = 0, 0
-        t1 = time.perf_counter()
-        while rows < 1 or (time.perf_counter() - t1 < gemm_budget_s and rows < 64):
-            r = rows % self.a_rows.shape[0]
-            o.gemm_mgrouped_full(self.a_rows[r:r + 1], np.ascontiguousarray(self.sa_rows[:, r:r + 1]),
-                                 wq, sw, np.array([0, 1], np.int32))
-            rows += 1
-            flops += 2 * self.wrows * K
-        t_gemm = time.perf_counter() - t1
-        desc = (f"fp64 GEMM of {rows} output rows x {self.wrows} cols x K={K} (expert {self.e}), "
-                f"permute+1x128 quantize of {self.ntok} tokens (top-{self.cfg.k}), 128x128 quantize "
-                f"and transpose of a [{self.wrows}x{K}] weight slab; 1 thread")
-        return flops / t_gemm / 1e12, self.q_bytes / t_quant / 1e9, desc
+    # ---- inputs (bf16 bits as uint16 host arrays)
+    @staticmethod
+    def _bits(t: torch.Tensor) -> np.ndarray:
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    def _rows(self, name, lo, hi):
+        c = self.cfg
+        if self.src is not None:
+            return self._bits(getattr(self.src, name)[lo:hi])
+        if name == "x":
+            return self._bits(W.gen_normal_bf16((hi - lo, c.hidden), W.SIGMA_X, c.seed, W.SID_X,
+                                                index_offset=lo * c.hidden))
+        return self._bits(W.gen_dy(c, row0=lo, rows=hi - lo))
+
+    def _weight(self, which, e, n0, n1):
+        """Rows [n0, n1) of expert e's weight, [1, n1 - n0, K]."""
+        c = self.cfg
+        N, K, sid = (c.n_up, c.hidden, W.SID_W_UP) if which == "up" else (c.hidden, c.inter, W.SID_W_DOWN)
+        if self.src is not None:
+            t = (self.src.w_up if which == "up" else self.src.w_down)[e:e + 1, n0:n1]
+            return self._bits(t)
+        return self._bits(W.gen_normal_bf16((1, n1 - n0, K), W.SIGMA_W, c.seed, sid,
+                                            index_offset=(e * N + n0) * K))
+
+    def _x_all(self):
+        if self._x is None:
+            self._x = self._rows("x", 0, self.cfg.T)
+        return self._x
+
+    # ---- units: (prepare() -> args, untimed; run(args) -> algorithmic amount)
+    def units(self, family):
+        c, o = self.cfg, self.o
+        T, K, k, E, R, N, I = c.T, c.hidden, c.k, c.E, c.R, c.n_up, c.inter
+        if family == "quant_act_permute":
+            slab = 64 if self.small else 512
+
+            def run(a):
+                o.quantize_act(a[0], a[1], E)
+                return bytes_route_quant(a[0].shape[0], K, k, E)
+            return [(lambda t0=t0: (self._rows("x", t0, min(T, t0 + slab)),
+                                    np.ascontiguousarray(self.ids[t0:t0 + slab])), run)
+                    for t0 in range(0, T, slab)]
+        if family == "quant_act_rows":
+            rows = 256 if self.small else 2048
+
+            def run(a):
+                o.quantize_act(a, None, 1)
+                return bytes_rows_quant(a.shape[0], N)
+            return [(lambda r0=r0: self._rows("dy", r0, min(R, r0 + rows)), run)
+                    for r0 in range(0, R, rows)]
+        if family == "quant_act_colwise":
+            offs, rt = self.route["offsets"], self.route["row_token"]
+
+            def prep(e):
+                o0, o1 = int(offs[e]), int(offs[e + 1])
+                if self.small:       # at most 128 rows of the expert (one token tile)
+                    o1 = min(o1, o0 + 128)
+                sub = np.array([0, o1 - o0], np.int32)
+                return (self._rows("dy", o0, o1), np.ascontiguousarray(self._x_all()[rt[o0:o1]]), sub)
+
+            def run(a):
+                o.quantize_act_colwise(a[0], a[2])
+                o.quantize_act_colwise(a[1], a[2])
+                pad = int((a[2][1] + 127) // 128 * 128)
+                return bytes_colwise(int(a[2][1]), N, pad) + bytes_colwise(int(a[2][1]), K, pad)
+            return [(lambda e=e: prep(e), run) for e in self.nz]
+
+        def slabs(which, rows_total):
+            step = 128 if self.small else rows_total
+            return [(e, n0, n0 + step) for e in range(E) for n0 in range(0, rows_total, step)]
+        if family == "quant_weight":
+            def run(a):
+                o.quantize_weight(a)
+                return bytes_weight_quant(1, a.shape[1], a.shape[2])
+            us = [(lambda u=u: self._weight("up", *u), run) for u in slabs("up", N)]
+            if I:
+                us += [(lambda u=u: self._weight("down", *u), run) for u in slabs("down", K)]
+            return us
+        if family == "transpose_blockq":
+            def run(a):
+                o.transpose_blockq(*a)
+                return bytes_transpose(1, a[0].shape[1], a[0].shape[2])
+            return [(lambda u=u: o.quantize_weight(self._weight("up", *u)), run)
+                    for u in slabs("up", N)]
+        raise ValueError(family)
+
+    def _gemm_setup(self):
+        """Operands of the up-projection GEMM for 64 rows of the largest
+        expert, quantized by the oracle (untimed, once)."""
+        if not hasattr(self, "_g"):
+            c, o = self.cfg, self.o
+            e = int(np.argmax(self.counts))
+            o0 = int(self.route["offsets"][e])
+            rows = self.route["row_token"][o0:o0 + 64]
+            xq = o.quantize_act(np.ascontiguousarray(self._x_all()[rows]), None, 1)
+            wq, sw = o.quantize_weight(self._weight("up", e, 0, c.n_up))
+            self._g = (xq["xq"], xq["sa"], wq, sw)
+        return self._g
+
+    def gemm_rate(self, nthreads, budget_s):
+        """fp64 oracle GEMM (all output columns of sampled rows): FLOP/s and rows."""
+        a, sa, wq, sw = self._gemm_setup()
+        N, K = wq.shape[1], wq.shape[2]
+        off = np.array([0, a.shape[0]], np.int32)
+        per = max(1, nthreads)
+        done, t0 = 0, time.perf_counter()
+        while done == 0 or time.perf_counter() - t0 < budget_s:
+            rows = np.arange(done, done + per) % a.shape[0]
+            r, cc = np.repeat(rows, N), np.tile(np.arange(N), per)
+            self.o.gemm_mgrouped_entries_threaded(a, sa, wq, sw, off, r, cc, nthreads=nthreads)
+            done += per
+        return 2.0 * done * N * K / (time.perf_counter() - t0), done
+
+    def time_1t(self, per_family=2, gemm_s=3.0):
+        """One thread: the first units of each family, and the GEMM rate."""
+        out, tot_b, tot_s = {}, 0.0, 0.0
+        for fam in self.FAMILIES:
+            us = self.units(fam)[:per_family]
+            b = s = 0.0
+            for prep, run in us:
+                a = prep()
+                t0 = time.perf_counter()
+                b += run(a)
+                s += time.perf_counter() - t0
+            out[fam] = {"gbs": b / s / 1e9, "units": len(us)}
+            tot_b, tot_s = tot_b + b, tot_s + s
+        g, rows = self.gemm_rate(1, gemm_s)
+        return {"threads": 1, "quantize_gbs": tot_b / tot_s / 1e9, "kernels": out,
+                "gemm_tflops": g / 1e12, "gemm_rows": rows}
+
+    def time_all(self, nthreads, budget_s=60.0, gemm_s=4.0, max_units=None, cache=None):
+        """`nthreads` threads over every family (budget_s / 5 seconds of timed
+        work each), then the GEMM rate on sampled rows (gemm_s seconds).
+        max_units caps the units per family; `cache` (a dict) keeps prepared
+        inputs between calls."""
+        from concurrent.futures import ThreadPoolExecutor
+        out, tot_b, tot_s = {}, 0.0, 0.0
+        share = budget_s / len(self.FAMILIES)
+        with ThreadPoolExecutor(max_workers=nthreads) as ex:
+            for fam in self.FAMILIES:
+                us = self.units(fam)
+                if max_units:
+                    us = us[:max_units]
+                b = s = 0.0
+                n_done = 0
+                while n_done < len(us):
+                    batch = us[n_done:n_done + 2 * nthreads]
+                    key = (fam, n_done)
+                    if cache is not None and key in cache:
+                        args = cache[key]
+                    else:
+                        args = list(ex.map(lambda u: u[0](), batch))
+                        if cache is not None:
+                            cache[key] = args
+                    t0 = time.perf_counter()
+                    b += sum(ex.map(lambda ua: ua[0][1](ua[1]), zip(batch, args)))
+                    s += time.perf_counter() - t0
+                    n_done += len(batch)
+                    if s > share:
+                        break
+                out[fam] = {"gbs": b / s / 1e9, "units": n_done, "of_units": len(us),
+                            "covered": n_done / len(self.units(fam))}
+                tot_b, tot_s = tot_b + b, tot_s + s
+        res = {"threads": nthreads, "quantize_gbs": tot_b / tot_s / 1e9, "kernels": out,
+               "covered": min(v["covered"] for v in out.values())}
+        if gemm_s > 0:
+            g, rows = self.gemm_rate(nthreads, gemm_s)
+            res.update(gemm_tflops=g / 1e12, gemm_rows=rows)
+        return res
+
+
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg: W.MoEConfig, source=None, budget_s: float = 60.0):
+    """The cpu_baseline object of the JSON line (oracle at 1 thread and at all
+    usable cores; `value` is the GEMM rate at all cores)."""
+    ob = OracleBaseline(cfg, source)
+    n = host_threads()
+    one = ob.time_1t()
+    allc = ob.time_all(n, budget_s=budget_s)
+    gemm_total = sum(a for b, a in work_of(cfg, padded_total_of(cfg))[0].values() if b == "tensor")
+    return {
+        "value": allc["gemm_tflops"], "unit": "TFLOP/s", "cores": n, "kind": "oracle",
+        "sample": (f"fp64 GEMM on {allc['gemm_rows']} sampled output rows (all {cfg.n_up} "
+                   f"columns, K={cfg.hidden}) at {n} threads; K1-K3 over "
+                   f"{100 * allc['covered']:.0f}% or more of the {cfg.name} workload at {n} "
+                   "threads; one-thread rates on the first units of each kernel"),
+        "quantize_gbs": allc["quantize_gbs"],
+        "threads_1": one, "threads_all": allc,
+        "gemm_full_step_s": {"value": gemm_total / (allc["gemm_tflops"] * 1e12),
+                             "extrapolated": True,
+                             "note": "the step's GEMM FLOPs over the sampled fp64 rate"},
+    }
 
 
 # --------------------------------------------------------------------------
@@ -538,30 +744,43 @@ def job_rate(world: int, units_per_rank: float, slowest_ms: float) -> float:
 
 
 def run_reference(args):
+    """The reference arm: the oracle on this host's cores (no GPU), each step a
+    bounded sample of the workload -- one unit per thread of every K1-K3
+    family (inputs prepared once) and a fixed time of the fp64 GEMM on
+    sampled rows.  Under torchrun only rank 0 runs and prints."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     cfg = W.CONFIGS[args.config]
-    sample = OracleSample(cfg)
+    ob = OracleBaseline(cfg)
+    n = host_threads()
+    cache = {}
     times, tf_list, gb_list = [], [], []
-    desc = ""
+    res = None
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        tf, gb, desc = sample.run(gemm_budget_s=2.0)
+        res = ob.time_all(n, budget_s=1e9, gemm_s=1.0, max_units=n, cache=cache)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
-            tf_list.append(tf)
-            gb_list.append(gb)
-    value = statistics.median(tf_list)
+            tf_list.append(res["gemm_tflops"])
+            gb_list.append(res["quantize_gbs"])
+    value = statistics.median(tf_list) if tf_list else res["gemm_tflops"]
+    desc = (f"per step: {n} units of each K1-K3 kernel of the {cfg.name} workload (token slabs, "
+            "row slabs, experts' token tiles, 128-row weight slabs) and 1 s of the fp64 GEMM on "
+            f"sampled output rows (all {cfg.n_up} columns, K={cfg.hidden}), at {n} threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "description": cfg.description},
-        "quantize_gbs": statistics.median(gb_list),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": desc},
+        "ms_per_step": 1e3 * statistics.median(times) if times else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "description": cfg.description, "E": cfg.E, "T": cfg.T,
+                   "k": cfg.k, "hidden": cfg.hidden, "n_up": cfg.n_up, "inter": cfg.inter,
+                   "routed_rows": cfg.R, "parallelism": f"oracle on {n} host threads"},
+        "quantize_gbs": statistics.median(gb_list) if gb_list else res["quantize_gbs"],
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": n, "kind": "oracle",
+                         "sample": desc, "quantize_gbs_by_kernel":
+                             {k_: v["gbs"] for k_, v in res["kernels"].items()}},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -581,11 +800,14 @@ def main():
     ap.add_argument("--impl", default="fg8", choices=["fg8", "reference"])
     ap.add_argument("--config", default="dsv3", choices=sorted(W.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=60.0,
+                    help="seconds of timed oracle work for the K1-K3 families of cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--fused-act", action="store_true",
-                    help="forward through the up-projection with the gated activation and its "
-                         "1x128 quantization fused in the epilogue (H comes from the up-projection "
-                         "instead of being a separate input)")
+    ap.add_argument("--unfused-act", action="store_true",
+                    help="forward through the plain up-projection (bf16 Y) and a separately "
+                         "generated, row-quantized down-projection input H, instead of the "
+                         "default up-projection with the gated activation and its 1x128 "
+                         "quantization fused in the epilogue")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -614,7 +836,7 @@ def main():
     fg8.lib()
 
     cfg = W.CONFIGS[args.config]
-    st = Step(cfg, dev, fused_act=args.fused_act)
+    st = Step(cfg, dev, fused_act=not args.unfused_act)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -693,27 +915,32 @@ def main():
                     "frac": tr_gb / pk["hbm_gbs"], "share": None,
                     "traffic": measured_traffic("transpose_blockq", cfg, st.padded_total),
                     "note": "not in the step: the step's WqT comes from the fused quantizer"})
-    # the fused up-projection + gated activation + 1x128 quantization on its own
-    # (outside the default step, which keeps the unfused chain)
-    if cfg.inter and not st.fused_act:
+    # the up-projection kernel that the step does not use, on its own and on
+    # the same operands: the plain one (bf16 Y) when the step runs the fused
+    # gated activation (the default), the fused one otherwise
+    if cfg.inter:
+        alt = "gemm_fprop_up" if st.fused_act else "gemm_fprop_up_swiglu_quant"
         with torch.cuda.stream(stream):
-            st.run_fused_up(stream)
+            st.run_up_alternative(stream)
             fu0, fu1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             fu0.record(stream)
             for _ in range(args.steps):
-                st.run_fused_up(stream)
+                st.run_up_alternative(stream)
             fu1.record(stream)
         torch.cuda.synchronize()
         fu_ms = fu0.elapsed_time(fu1) / args.steps
         fu_tf = 2.0 * cfg.R * cfg.n_up * cfg.hidden / (fu_ms * 1e-3) / 1e12
-        kernels.append({"kernel": "gemm_fprop_up_swiglu_quant", "standalone": True,
+        in_step = "gemm_fprop_up_swiglu_quant" if st.fused_act else "gemm_fprop_up"
+        kernels.append({"kernel": alt, "standalone": True,
                         "bound": "tensor", "ms": fu_ms, "achieved": fu_tf, "peak": fp8_peak,
                         "unit": "TFLOP/s", "frac": fu_tf / fp8_peak, "share": None,
-                        "traffic": measured_traffic("gemm_fprop_up_swiglu_quant", cfg, st.padded_total),
-                        "replaces_ms": kern_ms["gemm_fprop_up"],
-                        "note": "not in the step: replaces gemm_fprop_up (bf16 Y) and the row "
-                                "quantization of H; back-to-back launches, operands L2-warm "
-                                "only in part (W_up alone exceeds L2)"})
+                        "traffic": measured_traffic(alt, cfg, st.padded_total),
+                        "in_step_counterpart": in_step, "in_step_ms": kern_ms[in_step],
+                        "note": "not in the step: back-to-back launches on the step's operands "
+                                "(W_up alone exceeds L2); "
+                                + ("the fused kernel in the step replaces it and the row "
+                                   "quantization of H" if st.fused_act else
+                                   "it would replace gemm_fprop_up and the row quantization of H")})
     # unpermute + combine of the down-projection output on its own
     if cfg.inter:
         with torch.cuda.stream(stream):
@@ -816,9 +1043,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, gb, desc = OracleSample(cfg).run(gemm_budget_s=10.0)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc,
-               "quantize_gbs": gb}
+        cpu = cpu_baseline(cfg, st, budget_s=args.cpu_budget)
 
     if rank == 0:
         line = {

@@ -57,6 +57,7 @@ extern "C" const char* fg8_status_string(fg8_status s) {
         case FG8_ERR_CUDA: return "FG8_ERR_CUDA";
         case FG8_ERR_BAD_EXPERT_ID: return "FG8_ERR_BAD_EXPERT_ID";
         case FG8_ERR_TIMEOUT: return "FG8_ERR_TIMEOUT";
+        case FG8_ERR_WORKSPACE_SHARED: return "FG8_ERR_WORKSPACE_SHARED";
     }
     return "FG8_UNKNOWN_STATUS";
 }

@@ -47,8 +47,6 @@
 // wind down and TMEM is released); the kernel never traps.
 #include <cuda.h>
 
-#include <atomic>
-
 #include "fg8_common.cuh"
 #include "fg8_tma.cuh"
 
@@ -114,8 +112,8 @@ constexpr uint32_t kScaleSlotBytes = 4 * (BM + BN);            // 1536
 constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // contraction-grouped mode: tiles are handed out at run time.  The producer
-// takes the next tile number from a device counter (zeroed before the launch),
-// decodes it and publishes what the other roles need (K blocks, first output
+// takes the next tile number from a counter in the caller's workspace (zeroed
+// on the stream before the launch), decodes it and publishes what the other roles need (K blocks, first output
 // row and column) through a ring of kTileRing shared slots; the MMA thread and
 // the promotion warps read the ring.  Experts with few tokens are output-bound
 // (a 128 KB fp32 tile per 128x256 block) and experts with many are math-bound,
@@ -124,7 +122,12 @@ constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a
 // tiles share their A rows.
 constexpr int kTileRing = 8;
 constexpr int kMix = 4;
-constexpr int kCtrSlots = 64;   // launches that may run at the same time
+// Caller workspace of the contraction-grouped mode (zeroed before each launch):
+// word 0 is the tile ticket counter, word 1 counts the producers that have
+// finished, so the last one can check the ticket count (a workspace shared by
+// overlapping launches breaks it, and is reported instead of passing
+// unnoticed).
+constexpr size_t kGroupKWorkspace = 16;
 
 // shared memory map (offsets from a 1024-byte aligned base), per mode
 template <bool kGroupK>
@@ -133,8 +136,9 @@ struct Layout {
     static constexpr int kScaleSlots = kStages + 2;
     static constexpr uint32_t kOffStages = 0;
     static constexpr uint32_t kOffBars = kStages * kStageBytes;
-    // full, empty, tfull, tempty, drain (+ tile ring full / empty, contraction-grouped)
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kGroupK ? 2 * kTileRing : 2);
+    // full, empty, tfull, tempty, drain, then the tile ring (contraction-
+    // grouped) or the gate/up epilogue's exchange barriers (row-grouped)
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kGroupK ? 2 * kTileRing : 8);
     static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;   // tmem slot, abort flag
     static constexpr uint32_t kOffRing = align_up(kOffMisc + 16, 16);  // int4 [kTileRing]
     // row-grouped: tiles per expert, exclusive prefix; contraction-grouped:
@@ -146,8 +150,10 @@ struct Layout {
     static constexpr uint32_t kStageAll =
         Warps<kGroupK>::kEpiWarps * (kGroupK ? kTmaStagePerWarp : kStagePerWarp);
     static constexpr uint32_t kOffScales = kOffStage + kStageAll;
+    // contraction-grouped: the scale slots; row-grouped: the gate/up
+    // epilogue's row maxima, [TMEM buffer][warpgroup][row]
     static constexpr uint32_t kSmemBytes =
-        kOffScales + (kGroupK ? kScaleSlots * kScaleSlotBytes : 0) + 1024;   // + alignment slack
+        kOffScales + (kGroupK ? kScaleSlots * kScaleSlotBytes : 2 * 2 * BM * 4) + 1024;   // + alignment slack
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kOffStage % 16 == 0 && (kStageWords * 4) % 16 == 0, "16-byte staging");
 };
@@ -162,7 +168,7 @@ struct GemmArgs {
     int out_f32;
     void* out;
     int32_t* status;
-    unsigned int* tile_ctr;   // contraction-grouped: zeroed tile counter
+    unsigned int* ws;         // contraction-grouped: zeroed workspace words (see kGroupKWorkspace)
     // row-grouped gate/up mode: B holds [gate; up] (N = 2 I rows per expert),
     // out = E4M3 codes of h = silu(gate) * up [M_total][I], out_scale = their
     // 1x128 scales [I/128][M_total]
@@ -408,10 +414,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
-    // row-grouped gate/up epilogue: one exchange barrier per TMEM buffer (a
-    // buffer is reused only after the gate warps have released it, so an
-    // exchange can never complete twice before the gate warps see it)
-    auto xchg_bar = [&](uint32_t b) { return bar0 + 8u * (2 * kStages + 5 + b); };
+    // row-grouped gate/up epilogue: per TMEM buffer and warpgroup, one barrier
+    // for the half of the accumulators handed over and one for the row maxima
+    // (4 arrivals each).  A buffer is reused only after both warpgroups have
+    // released it, which they do after their waits, so no exchange barrier
+    // can complete twice before its waiters have seen it.
+    auto xchg_bar = [&](uint32_t b, int g) { return bar0 + 8u * (2 * kStages + 5 + 2 * b + g); };
+    auto amax_bar = [&](uint32_t b, int g) { return bar0 + 8u * (2 * kStages + 9 + 2 * b + g); };
     const uint32_t ring_full0 = bar0 + 8u * (2 * kStages + 5);
     const uint32_t ring_empty0 = ring_full0 + 8u * kTileRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -434,7 +443,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         mbar_init(drain_bar, 1);
         if (!kGroupK)
-            for (int b = 0; b < 2; ++b) mbar_init(xchg_bar(b), kEpiWarps / 2);
+            for (int b = 0; b < 2; ++b)
+                for (int g = 0; g < 2; ++g) {
+                    mbar_init(xchg_bar(b, g), kEpiWarps / 2);
+                    mbar_init(amax_bar(b, g), kEpiWarps / 2);
+                }
         if (kGroupK) {
             for (int i = 0; i < kTileRing; ++i) {
                 mbar_init(ring_full0 + 8u * i, 1);
@@ -502,7 +515,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         ok = false;
                         break;
                     }
-                    tile = (int)atomicAdd(a.tile_ctr, 1u);
+                    tile = (int)atomicAdd(a.ws, 1u);
                     if (tile >= total || tile < 0) {
                         ring_publish(ring, make_int4(-1, 0, 0, 0));
                         break;
@@ -604,6 +617,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint64_t t0 = fg8::globaltimer_ns();
             while (!mbar_try_wait(drain_bar, 0) && fg8::globaltimer_ns() - t0 < 100000000ull) {
             }
+
         }
       }
     } else {
@@ -617,7 +631,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int NB = a.N / 128, KBt = a.K / BK;
         uint32_t buf = 0, bphase = 0, sc = 0;
         uint32_t nbox = 0;    // TMA-store boxes issued by this warp (contraction-grouped)
-        uint32_t xphase = 0;  // gate/up epilogue: bit b = phase of xchg_bar(b)
+        uint32_t xphase = 0;  // gate/up epilogue: bit b = phase of buffer b's exchange barriers
         int e_hint = 0;
         bool ok = true;
         for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
@@ -757,74 +771,90 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             if (!ok) break;
             if (!kGroupK && kSwiglu) {
                 // Epilogue (gate/up): h = silu(gate) * up for this row's 128
-                // columns, quantized as one 1x128 tile.  The up warps park their
-                // accumulators in columns 128..255 of the last K block's TMEM
-                // buffer (same lanes), the gate warps read them back, form h and
-                // its codes and scale, and both release the buffer.
+                // columns, quantized as one 1x128 tile, the work split evenly:
+                // the gate warps form h for columns 0..63, the up warps for
+                // 64..127.  Each warpgroup parks the half of its accumulators
+                // the other needs in its own (already read) part of the last K
+                // block's TMEM buffer -- gate columns 64..127 at 64..127, up
+                // columns 0..63 at 128..191, same lanes -- and reads the other
+                // half back; the two row maxima meet through shared memory.
                 const uint32_t lbuf = buf ^ 1u;
-                const uint32_t xaddr = tmem_base + ((uint32_t)(32 * quarter) << 16) + lbuf * BN + 128;
-                if (grp == 1) {
-                    tmem_st64(xaddr, acc);
-                    tmem_st64(xaddr + 64, acc + 32);
-                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(xchg_bar(lbuf));
-                } else {
-                    // bounded wait for the four up warps of this tile
-                    if (!mbar_wait(xchg_bar(lbuf), (xphase >> lbuf) & 1u, abort_flag, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    xphase ^= 1u << lbuf;
-                    tc_fence_after();
-                    float amax = 0.f;
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        uint32_t u[64];
-                        tmem_ld64(xaddr + 64 * ch, u);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            float2& g = acc[32 * ch + i];
-                            g.x = silu_mul(g.x, __uint_as_float(u[2 * i]));
-                            g.y = silu_mul(g.y, __uint_as_float(u[2 * i + 1]));
-                            amax = fmaxf(amax, fmaxf(fabsf(g.x), fabsf(g.y)));
-                        }
-                    }
-                    const float sc = fg8::tile_scale(amax);
-                    const fg8::QScale q = fg8::make_qscale(sc);
-                    // 128 codes of this thread's row, 16 at a time, through the
-                    // warp's staging rows: each store writes 8 rows x 64 bytes
-                    uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kOffStage) + ep * 32 * kStageWords;
-                    uint4* my_row = reinterpret_cast<uint4*>(stg + lane * kStageWords);
-                    const int sub = ((lane >> 2) & 1) * 4 + (lane >> 3);
-                    const int quad = lane & 3;
-                    uint8_t* ob = static_cast<uint8_t*>(a.out) + col0 + 16 * quad;
-                    const int I = a.N / 2;
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll
-                        for (int w4 = 0; w4 < 4; ++w4) {
-                            uint2 c[2];
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const int base = 32 * ch + 8 * w4 + 4 * hh;   // float2 index: 8 values
-                                c[hh] = fg8::quant8f(acc[base], acc[base + 1], acc[base + 2], acc[base + 3], q);
-                            }
-                            my_row[w4] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
-                        }
-                        __syncwarp();
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const int rr = 8 * g + sub;
-                            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
-                            if (32 * quarter + rr < rows_valid)
-                                *reinterpret_cast<uint4*>(ob + (int64_t)(out_row0 + 32 * quarter + rr) * I + 64 * ch) = v;
-                        }
-                        __syncwarp();
-                    }
-                    if (row_ok) a.out_scale[(int64_t)(col0 / 128) * a.M_total + out_row0 + r] = sc;
+                const uint32_t lb = tmem_base + ((uint32_t)(32 * quarter) << 16) + lbuf * BN;
+                const uint32_t xp = (xphase >> lbuf) & 1u;
+                xphase ^= 1u << lbuf;
+                if (grp == 0)
+                    tmem_st64(lb + 64, acc + 32);
+                else
+                    tmem_st64(lb + 128, acc);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xchg_bar(lbuf, grp));
+                if (!mbar_wait(xchg_bar(lbuf, grp ^ 1), xp, abort_flag, a.status)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                float amax = 0.f;
+                // my 64 columns' h into acc[0..31]
+                if (grp == 0) {
+                    uint32_t u[64];
+                    tmem_ld64(lb + 128, u);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        acc[i].x = silu_mul(acc[i].x, __uint_as_float(u[2 * i]));
+                        acc[i].y = silu_mul(acc[i].y, __uint_as_float(u[2 * i + 1]));
+                        amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
+                    }
+                } else {
+                    uint32_t g[64];
+                    tmem_ld64(lb + 64, g);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        acc[i].x = silu_mul(__uint_as_float(g[2 * i]), acc[32 + i].x);
+                        acc[i].y = silu_mul(__uint_as_float(g[2 * i + 1]), acc[32 + i].y);
+                        amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
+                    }
+                }
+                float* s_amax = reinterpret_cast<float*>(smem + kOffScales) + (2 * lbuf) * BM;
+                s_amax[grp * BM + r] = amax;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(amax_bar(lbuf, grp));
+                if (!mbar_wait(amax_bar(lbuf, grp ^ 1), xp, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                amax = fmaxf(amax, s_amax[(grp ^ 1) * BM + r]);
+                const float sc = fg8::tile_scale(amax);
+                const fg8::QScale q = fg8::make_qscale(sc);
+                // 64 codes of this thread's row through the warp's staging rows:
+                // each store writes 8 rows x 64 bytes
+                uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kOffStage) + ep * 32 * kStageWords;
+                uint4* my_row = reinterpret_cast<uint4*>(stg + lane * kStageWords);
+                const int sub = ((lane >> 2) & 1) * 4 + (lane >> 3);
+                const int quad = lane & 3;
+                const int I = a.N / 2;
+                uint8_t* ob = static_cast<uint8_t*>(a.out) + col0 + 64 * grp + 16 * quad;
+#pragma unroll
+                for (int w4 = 0; w4 < 4; ++w4) {
+                    uint2 c[2];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int base = 8 * w4 + 4 * hh;   // float2 index: 8 values
+                        c[hh] = fg8::quant8f(acc[base], acc[base + 1], acc[base + 2], acc[base + 3], q);
+                    }
+                    my_row[w4] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int rr = 8 * g + sub;
+                    const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
+                    if (32 * quarter + rr < rows_valid)
+                        *reinterpret_cast<uint4*>(ob + (int64_t)(out_row0 + 32 * quarter + rr) * I) = v;
+                }
+                __syncwarp();
+                if (grp == 0 && row_ok) a.out_scale[(int64_t)(col0 / 128) * a.M_total + out_row0 + r] = sc;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tempty_bar(lbuf));
@@ -927,6 +957,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
     tc_fence_before();
     __syncthreads();
+    if (kGroupK && warp == 2 && lane == 0 && !*abort_flag) {
+        // Each producer took tickets until one was past the last tile, so after
+        // a clean launch the counter ends at tiles + CTAs.  The last CTA to get
+        // here checks it: another launch sharing the workspace leaves a
+        // different count.
+        __threadfence();
+        if (atomicAdd(a.ws + 1, 1u) == gridDim.x - 1) {
+            __threadfence();
+            const unsigned tiles = (unsigned)a.E * (unsigned)(a.M_total / BM) * (unsigned)((a.N + BN - 1) / BN);
+            if (*reinterpret_cast<volatile unsigned*>(a.ws) != tiles + gridDim.x)
+                fg8::set_status(a.status, FG8_ERR_WORKSPACE_SHARED);
+        }
+    }
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -945,32 +988,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
                                     box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// contraction-grouped tile counters (one per launch in flight, see kCtrSlots)
-__device__ unsigned int g_tile_ctr[kCtrSlots];
-std::atomic<void*> g_tile_ctr_addr[64];
-std::atomic<unsigned> g_tile_ctr_next{0};
-
-// A zeroed counter for one launch on `stream`, or nullptr on a CUDA error.
-unsigned int* take_tile_counter(cudaStream_t stream) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-    void* base = (dev >= 0 && dev < 64) ? g_tile_ctr_addr[dev].load() : nullptr;
-    if (base == nullptr) {
-        if (cudaGetSymbolAddress(&base, g_tile_ctr) != cudaSuccess) return nullptr;
-        if (dev >= 0 && dev < 64) g_tile_ctr_addr[dev].store(base);
-    }
-    unsigned int* ctr = static_cast<unsigned int*>(base) + g_tile_ctr_next.fetch_add(1) % kCtrSlots;
-    if (cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream) != cudaSuccess) return nullptr;
-    return ctr;
-}
-
 }  // namespace
+
+extern "C" size_t fg8_grouped_gemm_workspace(int group_mode) {
+    return group_mode == FG8_GROUP_K ? kGroupKWorkspace : 0;
+}
 
 extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const uint8_t* b,
                                        const float* sb, const int32_t* offsets, int64_t M_total,
                                        int N, int K, int E, int group_mode, int bscale_mode,
-                                       int out_dtype, void* out, int32_t* dev_status,
-                                       fg8_stream_t stream) {
+                                       int out_dtype, void* out, void* workspace, size_t ws_bytes,
+                                       int32_t* dev_status, fg8_stream_t stream) {
     if (!a || !sa || !b || !sb || !offsets || !out) return FG8_ERR_INVALID_ARG;
     if (E < 1 || N < 128 || K < 128 || N % 128 || K % 128 || M_total < 0)
         return FG8_ERR_INVALID_ARG;
@@ -997,6 +1025,8 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     } else if (group_mode == FG8_GROUP_K) {
         if (bscale_mode != FG8_BSCALE_ROW128) return FG8_ERR_UNSUPPORTED;
         if (M_total % 128 || !fg8h::aligned16(sa)) return FG8_ERR_INVALID_ARG;
+        if (!workspace || !fg8h::aligned16(workspace) || ws_bytes < kGroupKWorkspace)
+            return FG8_ERR_INVALID_ARG;
         if (out_dtype != FG8_OUT_F32) return FG8_ERR_UNSUPPORTED;
         if (M_total == 0) return FG8_OK;
         if ((int64_t)E * M_total > INT32_MAX) return FG8_ERR_UNSUPPORTED;
@@ -1036,12 +1066,13 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     args.out_f32 = out_dtype == FG8_OUT_F32;
     args.out = out;
     args.status = dev_status;
-    args.tile_ctr = nullptr;
+    args.ws = nullptr;
     args.swiglu = 0;
     args.out_scale = nullptr;
     if (group_mode == FG8_GROUP_K) {
-        args.tile_ctr = take_tile_counter((cudaStream_t)stream);
-        if (args.tile_ctr == nullptr) return FG8_ERR_CUDA;
+        args.ws = static_cast<unsigned int*>(workspace);
+        if (cudaMemsetAsync(workspace, 0, kGroupKWorkspace, (cudaStream_t)stream) != cudaSuccess)
+            return FG8_ERR_CUDA;
     }
     int64_t grid = fg8h::num_sms();
     if (grid > max_tiles) grid = max_tiles;
@@ -1092,7 +1123,7 @@ extern "C" fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const floa
     args.out_f32 = 0;
     args.out = hq;
     args.status = dev_status;
-    args.tile_ctr = nullptr;
+    args.ws = nullptr;
     args.swiglu = 1;
     args.out_scale = sh;
     int64_t grid = fg8h::num_sms();

@@ -23,7 +23,7 @@
 //    tokens).
 #include <cuda.h>
 
-#include <atomic>
+#include <mutex>
 
 #include "fg8_common.cuh"
 #include "fg8_tma.cuh"
@@ -561,7 +561,11 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
 // Host code cannot use the array's name as a device address (it is a host-side
 // stand-in), so on the first call on each device, with that device current,
 // the entry point asks the runtime for the array's device address and caches
-// it.  That first call should therefore come before any stream capture.
+// it, keyed by the unique id of the device's current context: if the context
+// is replaced (cudaDeviceReset, or the primary context released and created
+// again), the module is loaded anew, the array may move, and the next call
+// looks the address up again.  That first call (and the first after such a
+// replacement) should therefore come before any stream capture.
 
 namespace {
 
@@ -572,7 +576,58 @@ constexpr size_t kNoAllocScratchBytes =
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_noalloc_addr[kMaxDevices];
+struct NoallocCache {
+    unsigned long long ctx_id;   // unique id of the context the address belongs to
+    void* addr;
+};
+NoallocCache g_noalloc_cache[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the calling thread's current context (ids are never reused), or
+// 0 if there is none yet or the driver cannot tell.
+unsigned long long current_context_id() {
+    static const CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current device's current context.
+fg8_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FG8_ERR_CUDA;
+    const unsigned long long id = current_context_id();
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoallocCache& c = g_noalloc_cache[dev];
+    if (id != 0 && c.ctx_id == id && c.addr != nullptr) {
+        *out = c.addr;
+        return FG8_OK;
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return FG8_ERR_CUDA;
+    c.ctx_id = current_context_id();   // the lookup has made the context current
+    c.addr = p;
+    *out = p;
+    return FG8_OK;
+}
 
 }  // namespace
 
@@ -586,14 +641,9 @@ extern "C" fg8_status fg8_quantize_act_noalloc(const uint16_t* x, int64_t T, int
     size_t off_tot, off_chk;
     const size_t need = ws_layout(E, &off_tot, &off_chk);
     if (need > kNoAllocScratchBytes) return FG8_ERR_UNSUPPORTED;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FG8_ERR_CUDA;
-    void* scratch = g_noalloc_addr[dev].load(std::memory_order_acquire);
-    if (scratch == nullptr) {
-        if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr)
-            return FG8_ERR_CUDA;
-        g_noalloc_addr[dev].store(scratch, std::memory_order_release);
-    }
+    void* scratch = nullptr;
+    const fg8_status found = noalloc_scratch(&scratch);
+    if (found != FG8_OK) return found;
     // the permuting entry point clears the barrier word on every call; the
     // per-chunk counts and totals are fully written before they are read
     return fg8_quantize_act(x, T, K, topk_ids, k, E, nullptr, FG8_ROWWISE, xq, sa, row_token,

@@ -30,6 +30,7 @@ FG8_ERR_UNSUPPORTED = 2
 FG8_ERR_CUDA = 3
 FG8_ERR_BAD_EXPERT_ID = 4
 FG8_ERR_TIMEOUT = 5
+FG8_ERR_WORKSPACE_SHARED = 6
 FG8_ROWWISE = 1
 FG8_COLWISE = 2
 FG8_OUT_BF16 = 0
@@ -78,7 +79,10 @@ def lib() -> ctypes.CDLL:
         L.fg8_transpose_blockq.restype = _I
         L.fg8_transpose_blockq.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P]
         L.fg8_grouped_gemm.restype = _I
-        L.fg8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.fg8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _P,
+                                       _SZ, _P, _P]
+        L.fg8_grouped_gemm_workspace.restype = _SZ
+        L.fg8_grouped_gemm_workspace.argtypes = [_I]
         L.fg8_grouped_gemm_swiglu_quant.restype = _I
         L.fg8_grouped_gemm_swiglu_quant.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _P, _P,
                                                     _P, _P]
@@ -177,11 +181,15 @@ def fg8_transpose_blockq(wq, sw, E, N, K, wqT, swT, stream=None):
 
 
 def fg8_grouped_gemm(a, sa, b, sb, offsets, M_total, N, K, E, group_mode, bscale_mode,
-                     out_dtype, out, dev_status, stream=None):
+                     out_dtype, out, workspace, ws_bytes, dev_status, stream=None):
     _check(lib().fg8_grouped_gemm(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(offsets), M_total,
                                   N, K, E, group_mode, bscale_mode, out_dtype, _ptr(out),
-                                  _ptr(dev_status), _stream(stream)),
+                                  _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)),
            "fg8_grouped_gemm")
+
+
+def fg8_grouped_gemm_workspace(group_mode: int) -> int:
+    return int(lib().fg8_grouped_gemm_workspace(group_mode))
 
 
 def fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, sh, dev_status,
@@ -310,9 +318,10 @@ def transpose_blockq(wq: torch.Tensor, sw: torch.Tensor, stream=None):
 
 
 def grouped_gemm(a, sa, b, sb, offsets, out_dtype=FG8_OUT_BF16, group_mode=FG8_GROUP_M,
-                 dev_status=None, out=None, stream=None):
+                 dev_status=None, out=None, stream=None, workspace=None):
     """Row-grouped: a [M,K], b [E,N,K] -> out [M,N].  Contraction-grouped:
-    a [M,P], b [N,P] -> out [E,M,N]."""
+    a [M,P], b [N,P] -> out [E,M,N] (its tile counter lives in `workspace`,
+    allocated here when not given)."""
     M_total, K = a.shape
     E = offsets.numel() - 1
     if group_mode == FG8_GROUP_M:
@@ -326,8 +335,11 @@ def grouped_gemm(a, sa, b, sb, offsets, out_dtype=FG8_OUT_BF16, group_mode=FG8_G
     if out is None:
         dt = torch.float32 if out_dtype == FG8_OUT_F32 else torch.bfloat16
         out = torch.empty(shape, dtype=dt, device=a.device)
+    ws_bytes = fg8_grouped_gemm_workspace(group_mode)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=a.device)
     fg8_grouped_gemm(a, sa, b, sb, offsets, M_total, N, K, E, group_mode, bmode, out_dtype, out,
-                     dev_status, stream)
+                     workspace, ws_bytes if workspace is not None else 0, dev_status, stream)
     return out
 
 

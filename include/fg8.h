@@ -24,11 +24,11 @@
  * Conventions for every call:
  *  - All data pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, never synchronizes the stream and keeps no state
- *    between calls, so calls on different streams with disjoint buffers are
- *    independent, with two stated exceptions: the contraction-grouped GEMM's
- *    tile counters (fg8_grouped_gemm) and the allocation-free quantizer's
- *    scratch (fg8_quantize_act_noalloc) are device memory of the library.
- *    `stream` is a cudaStream_t (NULL = the legacy stream).
+ *    between calls, so calls on different streams with disjoint buffers
+ *    (workspaces included) are independent.  One stated exception: the
+ *    allocation-free quantizer's scratch (fg8_quantize_act_noalloc) is device
+ *    memory of the library.  `stream` is a cudaStream_t (NULL = the legacy
+ *    stream).
  *  - bf16 data is passed as uint16_t bit patterns.  FP8 data as uint8_t.
  *  - Calls are asynchronous.  Argument errors are found on the host and
  *    returned immediately (nothing is launched).  Launch failures return
@@ -56,7 +56,9 @@ typedef enum {
     FG8_ERR_UNSUPPORTED = 2,   /* valid but not implemented combination  */
     FG8_ERR_CUDA = 3,          /* a CUDA runtime/launch error            */
     FG8_ERR_BAD_EXPERT_ID = 4, /* device: an id outside [0, E) was met   */
-    FG8_ERR_TIMEOUT = 5        /* device: a bounded wait ran out         */
+    FG8_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out         */
+    FG8_ERR_WORKSPACE_SHARED = 6 /* device: a workspace was in use by an
+                                    overlapping call (results invalid)   */
 } fg8_status;
 
 typedef enum { FG8_ROWWISE = 1, FG8_COLWISE = 2 } fg8_act_layout;
@@ -131,10 +133,12 @@ fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
  *   nothing and calls no allocating routine.
  *   Limit: E <= 256; a larger E returns FG8_ERR_UNSUPPORTED.
  *   The first call on each device (with that device current) looks up the
- *   array's device address once; make that first call before any stream
- *   capture.  All calls on a device share the array: calls that overlap on
- *   the GPU race with each other.  The library resets what must start at zero
- *   on every call.
+ *   array's device address and keeps it for that device's context; the first
+ *   call after the context is replaced (cudaDeviceReset, or the primary
+ *   context released and created again) looks it up again.  Make those calls
+ *   before any stream capture.  All calls on a device share the array: calls
+ *   that overlap on the GPU race with each other.  The library resets what
+ *   must start at zero on every call.
  */
 fg8_status fg8_quantize_act_noalloc(const uint16_t* x, int64_t T, int64_t K,
                                     const int32_t* topk_ids, int k, int E,
@@ -205,7 +209,7 @@ fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N
  *            [offsets[e], offsets[e+1]); offsets[E] <= M_total
  *   out      [M_total][N] bf16 or fp32; rows outside [0, offsets[E]) are
  *            not written.  An expert with no rows costs nothing.
- *   N % 128 == 0, K % 128 == 0, E <= 1024.
+ *   N % 128 == 0, K % 128 == 0, E <= 1024.  workspace may be NULL.
  *
  * group_mode = FG8_GROUP_K (weight gradient; variable contraction per expert):
  *   a        E4M3 [M_total][K], sa fp32 [K/128][M_total]
@@ -218,10 +222,13 @@ fg8_status fg8_transpose_blockq(const uint8_t* wq, const float* sw, int E, int N
  *            sa and sb 16-byte aligned (the scale vectors are bulk-copied);
  *            out_dtype must be FG8_OUT_F32 (weight gradients are accumulated
  *            in fp32; other dtypes return FG8_ERR_UNSUPPORTED).
- *   The tiles are handed out at run time from a tile counter that the
- *   library keeps in device memory (64 per device, used in turn and zeroed
- *   on `stream` before each launch): at most 64 contraction-grouped launches
- *   may execute at the same time on one device.
+ *   The tiles are handed out at run time from a counter in `workspace`
+ *   (>= fg8_grouped_gemm_workspace(FG8_GROUP_K) bytes, 16-byte aligned,
+ *   zeroed by the call on `stream` before the launch).  Calls that share a
+ *   workspace must not overlap on the GPU; when they do, the tiles of a
+ *   launch are no longer processed exactly once, and the last CTA of the
+ *   launch reports FG8_ERR_WORKSPACE_SHARED in *dev_status (the output is
+ *   then invalid).
  *
  * The fp32 output is the accumulator; the bf16 output is its round-to-
  * nearest-even conversion.  dev_status may be NULL only if no device-side
@@ -232,7 +239,11 @@ fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa,
                             const uint8_t* b, const float* sb,
                             const int32_t* offsets, int64_t M_total, int N, int K, int E,
                             int group_mode, int bscale_mode, int out_dtype, void* out,
+                            void* workspace, size_t ws_bytes,
                             int32_t* dev_status, fg8_stream_t stream);
+
+/* Workspace bytes fg8_grouped_gemm needs in `group_mode` (0 for FG8_GROUP_M). */
+size_t fg8_grouped_gemm_workspace(int group_mode);
 
 /*
  * fg8_grouped_gemm_swiglu_quant -- the expert up-projection with its gated

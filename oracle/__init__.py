@@ -302,3 +302,177 @@ def gemm_kgrouped_entries(a, sa, b, sb, padoff, experts, rows, cols):
                                      M, N, P_cap, _ptr(experts), _ptr(rows), _ptr(cols),
                                      rows.size, _ptr(ref), _ptr(bound))
     return ref, bound
+
+
+# --------------------------------------------------------------------------
+# threaded drivers
+#
+# The same C functions as above, each called on disjoint slices of the input
+# from a pool of threads (ctypes releases the GIL for the duration of a call,
+# so the calls run in parallel).  Every thread runs the plain scalar loop of
+# the function it calls; the drivers only cut the work into independent pieces
+# (experts, rows or 128-column groups, which the method never couples) and
+# place each piece's results where the single call would have put them.
+# --------------------------------------------------------------------------
+
+def threads() -> int:
+    """Threads the drivers use: FG8_ORACLE_THREADS, else the usable cores."""
+    env = os.environ.get("FG8_ORACLE_THREADS")
+    if env:
+        return max(1, int(env))
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def _run(jobs, nthreads=None):
+    """Run the zero-argument callables `jobs` on a thread pool; re-raise errors."""
+    from concurrent.futures import ThreadPoolExecutor
+    n = nthreads or threads()
+    if n <= 1 or len(jobs) <= 1:
+        for j in jobs:
+            j()
+        return
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        for f in [ex.submit(j) for j in jobs]:
+            f.result()
+
+
+def _pieces(n: int, parts: int, quantum: int = 1):
+    """Split range(n) into at most `parts` contiguous pieces, boundaries on
+    multiples of `quantum`."""
+    units = (n + quantum - 1) // quantum
+    parts = max(1, min(parts, units))
+    cuts = [min(n, (units * i // parts) * quantum) for i in range(parts + 1)]
+    return [(cuts[i], cuts[i + 1]) for i in range(parts) if cuts[i + 1] > cuts[i]]
+
+
+def quantize_weight_threaded(w, nthreads=None):
+    """quantize_weight over expert slices (E > 1) or 128-row slabs (E == 1)."""
+    wu = _u16(w)
+    E, N, K = wu.shape
+    wq = np.zeros((E, N, K), np.uint8)
+    sw = np.zeros((E, N // 128, K // 128), np.float32)
+    n = nthreads or threads()
+    jobs = []
+    if E >= n:
+        for e0, e1 in _pieces(E, 4 * n):
+            jobs.append(lambda e0=e0, e1=e1: lib().fg8o_quantize_weight(
+                _ptr(wu[e0:e1]), e1 - e0, N, K, _ptr(wq[e0:e1]), _ptr(sw[e0:e1])))
+    else:
+        for e in range(E):
+            for n0, n1 in _pieces(N, 4 * n, 128):
+                jobs.append(lambda e=e, n0=n0, n1=n1: lib().fg8o_quantize_weight(
+                    _ptr(wu[e, n0:n1]), 1, n1 - n0, K, _ptr(wq[e, n0:n1]),
+                    _ptr(sw[e, n0 // 128:n1 // 128])))
+    _run(jobs, n)
+    return wq, sw
+
+
+def transpose_blockq_threaded(wq: np.ndarray, sw: np.ndarray, nthreads=None):
+    """transpose_blockq over expert slices."""
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    E, N, K = wq.shape
+    wqT = np.zeros((E, K, N), np.uint8)
+    swT = np.zeros((E, K // 128, N // 128), np.float32)
+    jobs = [lambda e=e: lib().fg8o_transpose_blockq(_ptr(wq[e]), _ptr(sw[e]), 1, N, K,
+                                                    _ptr(wqT[e]), _ptr(swT[e]))
+            for e in range(E)]
+    _run(jobs, nthreads)
+    return wqT, swT
+
+
+def quantize_rows_threaded(x, nthreads=None):
+    """Identity-mode quantize_act (rows already in expert order) over row slices:
+    returns (xq [R, K] u8, sa [K/128, R] f32)."""
+    xu = _u16(x)
+    R, K = xu.shape
+    xq = np.zeros((R, K), np.uint8)
+    sa = np.zeros((K // 128, R), np.float32)
+    n = nthreads or threads()
+
+    def job(r0, r1):
+        s = np.zeros((K // 128, r1 - r0), np.float32)
+        rt = np.full(r1 - r0, -1, np.int32)
+        tr = np.full(r1 - r0, -1, np.int32)
+        off = np.zeros(2, np.int32)
+        lib().fg8o_quantize_act_rowwise(_ptr(xu[r0:r1]), r1 - r0, K, None, 1, 1, _ptr(xq[r0:r1]),
+                                        _ptr(s), _ptr(rt), _ptr(tr), _ptr(off))
+        sa[:, r0:r1] = s
+    _run([lambda r0=r0, r1=r1: job(r0, r1) for r0, r1 in _pieces(R, 4 * n)], n)
+    return xq, sa
+
+
+def quantize_act_colwise_threaded(src, offsets: np.ndarray, row_map: np.ndarray | None = None,
+                                  P_cap: int | None = None, nthreads=None):
+    """quantize_act_colwise over groups of 128 columns (every column is
+    quantized on its own, so the groups are independent)."""
+    su = _u16(src)
+    C = su.shape[1]
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    E = offsets.size - 1
+    R = int(offsets[E])
+    if P_cap is None:
+        P_cap = colwise_capacity(R, E)
+    xqT = np.zeros((C, P_cap), np.uint8)
+    sT = np.zeros((P_cap // 128, C), np.float32)
+    padoff = np.zeros(E + 1, np.int32)
+    rm = None if row_map is None else np.ascontiguousarray(row_map, dtype=np.int32)
+    n = nthreads or threads()
+
+    def job(c0, c1):
+        part = np.ascontiguousarray(su[:, c0:c1])
+        s = np.zeros((P_cap // 128, c1 - c0), np.float32)
+        pad = np.zeros(E + 1, np.int32)
+        lib().fg8o_quantize_act_colwise(_ptr(part), c1 - c0, _ptr(rm), _ptr(offsets), E, P_cap,
+                                        _ptr(xqT[c0:c1]), _ptr(s), _ptr(pad))
+        sT[:, c0:c1] = s
+        if c0 == 0:
+            padoff[:] = pad
+    _run([lambda c0=c0, c1=c1: job(c0, c1) for c0, c1 in _pieces(C, 4 * n, 128)], n)
+    return dict(xqT=xqT, sT=sT, padoff=padoff)
+
+
+def gemm_mgrouped_entries_threaded(a, sa, b, sb, offsets, rows, cols, nthreads=None):
+    """gemm_mgrouped_entries over slices of the entry list."""
+    rows = np.ascontiguousarray(rows, np.int64)
+    cols = np.ascontiguousarray(cols, np.int64)
+    a = np.ascontiguousarray(a, np.uint8)
+    sa = np.ascontiguousarray(sa, np.float32)
+    b = np.ascontiguousarray(b, np.uint8)
+    sb = np.ascontiguousarray(sb, np.float32)
+    offsets = np.ascontiguousarray(offsets, np.int32)
+    M_total, K = a.shape
+    E, N, _ = b.shape
+    ref = np.zeros(rows.size, np.float64)
+    bound = np.zeros(rows.size, np.float64)
+    n = nthreads or threads()
+    jobs = [lambda i0=i0, i1=i1: lib().fg8o_gemm_mgrouped_entries(
+        _ptr(a), _ptr(sa), M_total, _ptr(b), _ptr(sb), _ptr(offsets), E, N, K,
+        _ptr(rows[i0:i1]), _ptr(cols[i0:i1]), i1 - i0, _ptr(ref[i0:i1]), _ptr(bound[i0:i1]))
+        for i0, i1 in _pieces(rows.size, 4 * n)]
+    _run(jobs, n)
+    return ref, bound
+
+
+def gemm_dense_fp64(a, sa, b, sb):
+    """All entries of the single-group product (E = 1) and their |term| sums:
+        out[r][n] = sum_k dq(a[r][k]) sa[k/128][r] * dq(b[n][k]) sb[n/128][k/128]
+    written as one fp64 matrix product of the dequantized operands (numpy's
+    matmul is the library step).  Every dequantized operand is exact in fp64
+    (a 4-bit code times a 24-bit scale); the products and the sum round at
+    2^-53, far below the GEMM tolerance.
+
+    a u8 [M, K], sa f32 [K/128, M], b u8 [N, K] (or [1, N, K]), sb f32
+    [N/128, K/128] (or [1, ...]).  Returns (ref fp64 [M, N], bound fp64 [M, N]).
+    """
+    a = np.ascontiguousarray(a, np.uint8)
+    b = np.ascontiguousarray(b, np.uint8).reshape(-1, a.shape[1])
+    sa = np.asarray(sa, np.float32)
+    sb = np.asarray(sb, np.float32).reshape(b.shape[0] // 128, a.shape[1] // 128)
+    dq = e4m3_decode_table()
+    A = dq[a] * np.repeat(sa.T.astype(np.float64), 128, axis=1)
+    B = dq[b] * np.repeat(np.repeat(sb.astype(np.float64), 128, axis=0), 128, axis=1)
+    return A @ B.T, np.abs(A) @ np.abs(B).T

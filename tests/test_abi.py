@@ -56,19 +56,28 @@ def test_null_and_shape_arguments_rejected_on_host(L):
     assert L.fg8_transpose_blockq(None, None, 1, 128, 128, None, None, None) == INV
     assert L.fg8_transpose_blockq(16, 16, 1, 128, 130, 16, 16, None) == INV  # K % 128
     assert L.fg8_grouped_gemm(None, None, None, None, None, 128, 128, 128, 1, 0, 0, 0, None,
-                              None, None) == INV
-    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 0, 0, 7, 16, None,
+                              None, 0, None, None) == INV
+    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 0, 0, 7, 16, None, 0, None,
                               None) == INV                                    # out dtype
+    # contraction-grouped: the tile counter's workspace is required, aligned, large enough
+    need = fg8.fg8_grouped_gemm_workspace(fg8.FG8_GROUP_K)
+    assert need >= 12 and fg8.fg8_grouped_gemm_workspace(fg8.FG8_GROUP_M) == 0
+    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 1, 1, 1, 16, None, need, None,
+                              None) == INV
+    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 1, 1, 1, 16, 16, need - 1,
+                              None, None) == INV
+    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 1, 1, 1, 16, 20, need, None,
+                              None) == INV
     assert L.fg8_quantize_act(None, 10, 128, None, 1, 1, None, 1, 16, 16, None, None, None,
                               None, None, None, 0, None, None) == INV         # x null
     assert L.fg8_quantize_act(16, 10, 100, None, 1, 1, None, 1, 16, 16, None, None, None,
                               None, None, None, 0, None, None) == INV         # K % 128
     # misaligned FP8 / bf16 buffers
     assert L.fg8_quantize_weight(18, 1, 128, 128, 16, 16, None, None) == INV
-    assert L.fg8_grouped_gemm(17, 16, 16, 16, 16, 128, 128, 128, 1, 0, 0, 0, 16, None,
+    assert L.fg8_grouped_gemm(17, 16, 16, 16, 16, 128, 128, 128, 1, 0, 0, 0, 16, None, 0, None,
                               None) == INV
     # unsupported combinations
-    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 0, 1, 0, 16, None,
+    assert L.fg8_grouped_gemm(16, 16, 16, 16, 16, 128, 128, 128, 1, 0, 1, 0, 16, None, 0, None,
                               None) == fg8.FG8_ERR_UNSUPPORTED               # M-grouped + row scales
     assert L.fg8_quantize_act(16, 10, 128, 16, 33, 4, None, 1, 16, 16, 16, 16, 16, None, None,
                               16, 1 << 20, None, None) == fg8.FG8_ERR_UNSUPPORTED  # k > 32

@@ -313,30 +313,34 @@ def test_gemm_kgrouped_interleaved_order_full(oracle):
         check(got[e].ravel(), ref, bound, f"interleaved expert {e}")
 
 
-def test_gemm_kgrouped_tile_counters_reused_and_concurrent():
-    """The contraction-grouped GEMM hands out tiles from library-held counters
-    (64, used in turn).  70 launches on one stream wrap around them, and pairs
-    of launches on two streams run at the same time; every result must equal
-    the first bit for bit (the kernel is deterministic)."""
+def test_gemm_kgrouped_workspaces_reused_and_concurrent():
+    """The contraction-grouped GEMM hands out tiles from a counter in the
+    caller's workspace.  One workspace reused by 10 launches in a row on one
+    stream, and 72 launches spread over 4 streams with a workspace each (more
+    than any fixed pool of counters would hold), must all equal the first
+    result bit for bit (the kernel is deterministic) with a clean status."""
     counts = [5, 300, 0, 129, 77, 256, 1, 40]
     M, N = 128, 256
     padoff, a, b, sa, sb = _kgrouped_operands(counts, M, N, 33)
     args = [t.cuda() for t in (a, sa, b, sb)] + [torch.from_numpy(padoff).cuda()]
+    need = fg8.fg8_grouped_gemm_workspace(fg8.FG8_GROUP_K)
     st = fg8.new_status()
 
-    def run(stream=None):
+    def run(ws, stream=None):
         return fg8.grouped_gemm(*args, out_dtype=fg8.FG8_OUT_F32, group_mode=fg8.FG8_GROUP_K,
-                                dev_status=st, stream=stream)
+                                dev_status=st, stream=stream, workspace=ws)
 
-    first = run()
+    ws0 = torch.empty(need, dtype=torch.uint8, device="cuda")
+    first = run(ws0)
     torch.cuda.synchronize()
-    outs = [run() for _ in range(70)]
-    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
-    for _ in range(4):
-        with torch.cuda.stream(s1):
-            outs.append(run(s1.cuda_stream))
-        with torch.cuda.stream(s2):
-            outs.append(run(s2.cuda_stream))
+    outs = [run(ws0) for _ in range(10)]
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    wss = [torch.empty(need, dtype=torch.uint8, device="cuda") for _ in range(72)]
+    torch.cuda.synchronize()
+    for i, ws in enumerate(wss):
+        s_ = streams[i % 4]
+        with torch.cuda.stream(s_):
+            outs.append(run(ws, s_.cuda_stream))
     torch.cuda.synchronize()
     assert st.item() == 0
     for o in outs:

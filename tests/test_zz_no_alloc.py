@@ -3,9 +3,12 @@
 It is meant for callers that cannot allocate device memory (a plugin whose
 host framework owns all allocations, or a path that must not enter the
 allocator): its scratch is an array inside the library.  This test calls it
-through the C ABI twice in a row and checks each result against the regular
-entry point, fg8_quantize_act, which uses a caller-provided workspace.  Both
-results must agree bit for bit, like every quantizer comparison here.
+through the C ABI twice in a row and checks each result bit for bit against
+the oracle (the routing maps and the 1x128 codes and scales of every routed
+row) and against the regular entry point, fg8_quantize_act, which uses a
+caller-provided workspace.  The cases include an expert count that is not a
+multiple of 64, so the scratch layout's rounding is exercised at the array's
+end (E = 255 of at most 256).
 
 The file is named so that pytest collects it last."""
 
@@ -40,19 +43,35 @@ def _noalloc(x, ids, E):
     return out
 
 
-@pytest.mark.parametrize("name", ["tiny", "dsv3"])
-def test_noalloc_matches_workspace_entry_point_twice(name):
+def _case(name):
+    if name == "E255":
+        T, K, E, k = 777, 512, 255, 8
+        rng = np.random.default_rng(255)
+        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+        return W.gen_normal_bf16((T, K), 1.0, 255, 1), ids, E
+    cfg = W.CONFIGS[name]
+    return W.gen_x(cfg), W.route(cfg), cfg.E
+
+
+@pytest.mark.parametrize("name", ["tiny", "E255", "dsv3"])
+def test_noalloc_matches_oracle_and_workspace_entry_point_twice(oracle, name):
     fbuild.build()
     fg8.lib()
-    cfg = W.CONFIGS[name]
-    x = W.gen_x(cfg, device="cuda")
-    ids = torch.from_numpy(W.route(cfg)).cuda()
-    ref = fg8.quantize_act(x, ids, cfg.E)
+    x_cpu, ids_np, E = _case(name)
+    x = x_cpu.cuda()
+    ids = torch.from_numpy(ids_np).cuda()
+    r = oracle.route(ids_np, E)
+    q = oracle.quantize_act(x_cpu, None, 1)          # each token row, 1x128 tiles
+    rt = r["row_token"]
+    expect = dict(xq=q["xq"][rt], sa=q["sa"][:, rt], row_token=rt, token_row=r["token_row"],
+                  offsets=r["offsets"])
+    ref = fg8.quantize_act(x, ids, E)
     for _ in range(2):
-        got = _noalloc(x, ids, cfg.E)
+        got = _noalloc(x, ids, E)
         torch.cuda.synchronize()
         assert got["status"].item() == 0 and ref["status"].item() == 0
         for key in ("xq", "sa", "row_token", "token_row", "offsets"):
+            assert np.array_equal(got[key].cpu().numpy(), expect[key]), key
             assert torch.equal(got[key], ref[key]), key
 
 
