@@ -26,6 +26,7 @@
 #include <mutex>
 
 #include "fg8_common.cuh"
+#include "fg8_route.cuh"
 #include "fg8_tma.cuh"
 
 namespace {
@@ -127,33 +128,32 @@ struct RouteArgs {
     int32_t* totals;        // workspace: [E]
     int32_t* chunk_counts;  // workspace: [gridDim.x][E]
     int32_t* status;
+    // fused routing (fg8_route_quantize_act): the ids are produced by the
+    // kernel itself from router logits and the per-expert bias
+    const float* logits;
+    const float* bias;
+    int32_t* ids_out;
+    float* affinity;
 };
 
-__global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
-    __shared__ int32_t s_cnt[kMaxE];
-    __shared__ int32_t s_off[kMaxE + 1];
-    __shared__ int32_t s_warp[33];
+// Shared memory of the permuting kernels.
+struct RouteSmem {
+    int32_t cnt[kMaxE];
+    int32_t off[kMaxE + 1];
+    int32_t warp[33];
+};
 
+// Phases B and C of the permuting kernels, after every CTA has written its
+// chunk histogram to a.chunk_counts and passed the first grid barrier.
+__device__ __forceinline__ void route_quant_scan_place_quantize(const RouteArgs& a, RouteSmem& sm) {
     const int G = gridDim.x, c = blockIdx.x, t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
     const int E = a.E, k = a.k;
     const int64_t t_begin = (int64_t)c * a.T / G, t_end = (int64_t)(c + 1) * a.T / G;
     const int64_t p_begin = t_begin * k, p_end = t_end * k;
     const int64_t R = a.T * k;
-
-    // ---- phase A: chunk histogram
-    for (int e = t; e < E; e += kThreads) s_cnt[e] = 0;
-    __syncthreads();
-    for (int64_t p = p_begin + t; p < p_end; p += kThreads) {
-        const int32_t e = a.ids[p];
-        if (e >= 0 && e < E)
-            atomicAdd(&s_cnt[e], 1);
-        else
-            fg8::set_status(a.status, FG8_ERR_BAD_EXPERT_ID);
-    }
-    __syncthreads();
-    for (int e = t; e < E; e += kThreads) a.chunk_counts[(int64_t)c * E + e] = s_cnt[e];
-    if (!fg8::grid_barrier(a.bar, (uint32_t)G, a.status)) return;
+    int32_t* s_cnt = sm.cnt;
+    int32_t* s_off = sm.off;
 
     // ---- phase B: per expert, exclusive scan over chunks (one warp each)
     for (int e = c * kWarps + warp; e < E; e += G * kWarps) {
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
     // ---- phase C: offsets, stable ranks, index maps
     for (int e = t; e < E; e += kThreads) s_cnt[e] = a.totals[e];
     __syncthreads();
-    fg8::block_exclusive_scan(s_cnt, s_off, E, s_warp);
+    fg8::block_exclusive_scan(s_cnt, s_off, E, sm.warp);
     if (c == 0)
         for (int e = t; e <= E; e += kThreads) a.offsets_out[e] = s_off[e];
     // s_cnt becomes this chunk's next free row per expert
@@ -210,6 +210,66 @@ __global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
         const int my_row = lane < k ? a.token_row[tok * k + lane] : -1;
         quant_row(a.x + tok * a.K, a.K, my_row, k, a.xq, a.sa, R, lane);
     }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) route_quant(RouteArgs a) {
+    __shared__ RouteSmem sm;
+    const int G = gridDim.x, c = blockIdx.x, t = threadIdx.x;
+    const int E = a.E, k = a.k;
+    const int64_t t_begin = (int64_t)c * a.T / G, t_end = (int64_t)(c + 1) * a.T / G;
+
+    // ---- phase A: chunk histogram of the given ids
+    for (int e = t; e < E; e += kThreads) sm.cnt[e] = 0;
+    __syncthreads();
+    for (int64_t p = t_begin * k + t; p < t_end * k; p += kThreads) {
+        const int32_t e = a.ids[p];
+        if (e >= 0 && e < E)
+            atomicAdd(&sm.cnt[e], 1);
+        else
+            fg8::set_status(a.status, FG8_ERR_BAD_EXPERT_ID);
+    }
+    __syncthreads();
+    for (int e = t; e < E; e += kThreads) a.chunk_counts[(int64_t)c * E + e] = sm.cnt[e];
+    if (!fg8::grid_barrier(a.bar, (uint32_t)G, a.status)) return;
+    route_quant_scan_place_quantize(a, sm);
+}
+
+// Routing fused in front of the permute: phase A routes this CTA's tokens
+// (sigmoid affinity + bias, top-k, one warp per token, DeepSeek-V3 summary
+// sec. 2.1), writes their ids and affinities and histograms the chosen
+// experts in the same pass; phases B and C are those of route_quant (phase C
+// reads back the ids this CTA has just written).  PER_LANE * 32 >= E.
+template <int PER_LANE>
+__global__ void __launch_bounds__(kThreads, PER_LANE >= 16 ? 1 : 2) route_topk_quant(RouteArgs a) {
+    __shared__ RouteSmem sm;
+    const int G = gridDim.x, c = blockIdx.x, t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5;
+    const int E = a.E, k = a.k;
+    const int64_t t_begin = (int64_t)c * a.T / G, t_end = (int64_t)(c + 1) * a.T / G;
+
+    // ---- phase A: route the chunk's tokens, histogram the choices
+    for (int e = t; e < E; e += kThreads) sm.cnt[e] = 0;
+    float bl[PER_LANE];
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+        const int e = lane + 32 * i;
+        bl[i] = e < E ? a.bias[e] : 0.f;
+    }
+    __syncthreads();
+    for (int64_t tok = t_begin + warp; tok < t_end; tok += kWarps) {
+        int32_t id;
+        float sv;
+        fg8::route_token<PER_LANE>(a.logits + tok * E, bl, E, k, lane, id, sv);
+        if (lane < k) {
+            a.ids_out[tok * k + lane] = id;
+            a.affinity[tok * k + lane] = sv;
+            atomicAdd(&sm.cnt[id], 1);
+        }
+    }
+    __syncthreads();
+    for (int e = t; e < E; e += kThreads) a.chunk_counts[(int64_t)c * E + e] = sm.cnt[e];
+    if (!fg8::grid_barrier(a.bar, (uint32_t)G, a.status)) return;
+    route_quant_scan_place_quantize(a, sm);
 }
 
 // --------------------------------------------------------------------------
@@ -426,6 +486,34 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
     }
 }
 
+size_t ws_layout(int64_t E, size_t* off_totals, size_t* off_chunks);
+inline void ws_layout_fwd(int64_t E, size_t* a, size_t* b) { ws_layout(E, a, b); }
+
+// Cooperative launch of a permuting kernel (all CTAs resident: its grid
+// barriers need that) on the workspace; the barrier word is cleared first.
+fg8_status launch_permuting(const void* kern, RouteArgs& a, void* workspace, cudaStream_t st) {
+    size_t off_tot, off_chk;
+    ws_layout_fwd(a.E, &off_tot, &off_chk);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
+        per_sm < 1)
+        return FG8_ERR_CUDA;
+    int64_t G = (int64_t)per_sm * fg8h::num_sms();
+    if (G > kMaxGrid) G = kMaxGrid;
+    if (G > (a.T + 1) / 2) G = (a.T + 1) / 2;
+    if (G < 1) G = 1;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return FG8_ERR_CUDA;
+    a.bar = reinterpret_cast<uint32_t*>(ws);
+    a.totals = reinterpret_cast<int32_t*>(ws + off_tot);
+    a.chunk_counts = reinterpret_cast<int32_t*>(ws + off_chk);
+    void* args[] = {&a};
+    if (cudaLaunchCooperativeKernel(kern, dim3((unsigned)G), dim3(kThreads), args, 0, st) !=
+        cudaSuccess)
+        return FG8_ERR_CUDA;
+    return fg8h::launch_status();
+}
+
 size_t ws_layout(int64_t E, size_t* off_totals, size_t* off_chunks) {
     const size_t bar = 256;                                       // barrier counter(s)
     const size_t totals = ((size_t)E * 4 + 255) / 256 * 256;
@@ -498,29 +586,12 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
         size_t off_tot, off_chk;
         const size_t need = ws_layout(E, &off_tot, &off_chk);
         if (ws_bytes < need) return FG8_ERR_INVALID_ARG;
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_quant, kThreads, 0) !=
-                cudaSuccess || per_sm < 1)
-            return FG8_ERR_CUDA;
-        int64_t G = (int64_t)per_sm * fg8h::num_sms();
-        if (G > kMaxGrid) G = kMaxGrid;
-        if (G > (T + 1) / 2) G = (T + 1) / 2;
-        if (G < 1) G = 1;
-        uint8_t* ws = static_cast<uint8_t*>(workspace);
-        if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return FG8_ERR_CUDA;
-        RouteArgs a;
+        RouteArgs a = {};
         a.x = x; a.T = T; a.K = K; a.ids = topk_ids; a.k = k; a.E = E;
         a.xq = xq; a.sa = sa; a.row_token = row_token; a.token_row = token_row;
         a.offsets_out = offsets_out;
-        a.bar = reinterpret_cast<uint32_t*>(ws);
-        a.totals = reinterpret_cast<int32_t*>(ws + off_tot);
-        a.chunk_counts = reinterpret_cast<int32_t*>(ws + off_chk);
         a.status = dev_status;
-        void* args[] = {&a};
-        if (cudaLaunchCooperativeKernel((const void*)route_quant, dim3((unsigned)G), dim3(kThreads),
-                                        args, 0, st) != cudaSuccess)
-            return FG8_ERR_CUDA;
-        return fg8h::launch_status();
+        return launch_permuting((const void*)route_quant, a, workspace, st);
     }
 
     if (layout == FG8_COLWISE) {
@@ -544,6 +615,43 @@ extern "C" fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
         return fg8h::launch_status();
     }
     return FG8_ERR_INVALID_ARG;
+}
+
+extern "C" fg8_status fg8_route_quantize_act(const float* logits, const float* bias,
+                                             const uint16_t* x, int64_t T, int64_t K, int k, int E,
+                                             int32_t* topk_ids, float* affinity, uint8_t* xq,
+                                             float* sa, int32_t* row_token, int32_t* token_row,
+                                             int32_t* offsets_out, void* workspace, size_t ws_bytes,
+                                             int32_t* dev_status, fg8_stream_t stream) {
+    cudaStream_t st = (cudaStream_t)stream;
+    if (T < 0 || K < 128 || K % 128 || E < 1 || E > 1024 || k < 1 || k > fg8::kRouteMaxK || k > E)
+        return FG8_ERR_INVALID_ARG;
+    if (!offsets_out) return FG8_ERR_INVALID_ARG;
+    if (T == 0)
+        return cudaMemsetAsync(offsets_out, 0, sizeof(int32_t) * ((size_t)E + 1), st) == cudaSuccess
+                   ? FG8_OK : FG8_ERR_CUDA;
+    if (!logits || !bias || !x || !topk_ids || !affinity || !xq || !sa || !row_token ||
+        !token_row || !workspace)
+        return FG8_ERR_INVALID_ARG;
+    if (!fg8h::aligned16(x) || !fg8h::aligned16(xq) || !fg8h::aligned16(workspace) ||
+        ((reinterpret_cast<uintptr_t>(logits) | reinterpret_cast<uintptr_t>(bias) |
+          reinterpret_cast<uintptr_t>(affinity) | reinterpret_cast<uintptr_t>(sa)) & 3))
+        return FG8_ERR_INVALID_ARG;
+    if (T * k > (int64_t)INT32_MAX || T > INT64_MAX / E) return FG8_ERR_UNSUPPORTED;
+    size_t off_tot, off_chk;
+    if (ws_bytes < ws_layout(E, &off_tot, &off_chk)) return FG8_ERR_INVALID_ARG;
+    RouteArgs a = {};
+    a.x = x; a.T = T; a.K = K; a.ids = topk_ids; a.k = k; a.E = E;
+    a.xq = xq; a.sa = sa; a.row_token = row_token; a.token_row = token_row;
+    a.offsets_out = offsets_out;
+    a.status = dev_status;
+    a.logits = logits; a.bias = bias; a.ids_out = topk_ids; a.affinity = affinity;
+    const void* kern = E <= 64    ? (const void*)route_topk_quant<2>
+                       : E <= 128 ? (const void*)route_topk_quant<4>
+                       : E <= 256 ? (const void*)route_topk_quant<8>
+                       : E <= 512 ? (const void*)route_topk_quant<16>
+                                  : (const void*)route_topk_quant<32>;
+    return launch_permuting(kern, a, workspace, st);
 }
 
 // --------------------------------------------------------------------------

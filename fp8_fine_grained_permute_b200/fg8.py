@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.fg8_quantize_act.restype = _I
         L.fg8_quantize_act.argtypes = [_P, _I64, _I64, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _SZ, _P, _P]
+        L.fg8_route_quantize_act.restype = _I
+        L.fg8_route_quantize_act.argtypes = [_P, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _P, _P,
+                                             _P, _P, _P, _SZ, _P, _P]
         L.fg8_quantize_act_noalloc.restype = _I
         L.fg8_quantize_act_noalloc.argtypes = [_P, _I64, _I64, _P, _I, _I, _P, _P, _P, _P, _P,
                                                _P, _P]
@@ -90,6 +93,12 @@ def lib() -> ctypes.CDLL:
         L.fg8_route_topk.argtypes = [_P, _P, _I64, _I, _I, _P, _P, _P]
         L.fg8_unpermute_combine.restype = _I
         L.fg8_unpermute_combine.argtypes = [_P, _I64, _I, _P, _P, _I64, _I, _I, _I, _P, _P]
+        L.fg8_ep_pack_scales.restype = _I
+        L.fg8_ep_pack_scales.argtypes = [_P, _I64, _I64, _P, _P]
+        L.fg8_ep_unpack.restype = _I
+        L.fg8_ep_unpack.argtypes = [_P, _P, _P, _I, _I, _I64, _I64, _P, _P, _P, _P, _P, _P]
+        L.fg8_gather_rows.restype = _I
+        L.fg8_gather_rows.argtypes = [_P, _I64, _I64, _P, _I64, _P, _P, _P]
         L.fg8_selftest_wait_timeout.restype = _I
         L.fg8_selftest_wait_timeout.argtypes = [_I, _P, _P, _P]
         L.fg8_status_string.restype = ctypes.c_char_p
@@ -142,6 +151,16 @@ def fg8_quantize_act(x, T, K, topk_ids, k, E, offsets_in, layout, xq, sa, row_to
                                   _ptr(offsets_out), _ptr(xqT), _ptr(saT), _ptr(workspace),
                                   ws_bytes, _ptr(dev_status), _stream(stream)),
            "fg8_quantize_act")
+
+
+def fg8_route_quantize_act(logits, bias, x, T, K, k, E, topk_ids, affinity, xq, sa, row_token,
+                           token_row, offsets_out, workspace, ws_bytes, dev_status, stream=None):
+    _check(lib().fg8_route_quantize_act(_ptr(logits), _ptr(bias), _ptr(x), T, K, k, E,
+                                        _ptr(topk_ids), _ptr(affinity), _ptr(xq), _ptr(sa),
+                                        _ptr(row_token), _ptr(token_row), _ptr(offsets_out),
+                                        _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                        _stream(stream)),
+           "fg8_route_quantize_act")
 
 
 def fg8_quantize_act_noalloc(x, T, K, topk_ids, k, E, xq, sa, row_token, token_row, offsets_out,
@@ -213,6 +232,25 @@ def fg8_unpermute_combine(y, R, C, token_row, affinity, T, k, normalize, out_dty
            "fg8_unpermute_combine")
 
 
+def fg8_ep_pack_scales(sa, R, K, sa_rows, stream=None):
+    _check(lib().fg8_ep_pack_scales(_ptr(sa), R, K, _ptr(sa_rows), _stream(stream)),
+           "fg8_ep_pack_scales")
+
+
+def fg8_ep_unpack(recv_xq, recv_sa, counts, W, E_loc, R_recv, K, xq, sa, offsets, recv_to_local,
+                  dev_status, stream=None):
+    _check(lib().fg8_ep_unpack(_ptr(recv_xq), _ptr(recv_sa), _ptr(counts), W, E_loc, R_recv, K,
+                               _ptr(xq), _ptr(sa), _ptr(offsets), _ptr(recv_to_local),
+                               _ptr(dev_status), _stream(stream)),
+           "fg8_ep_unpack")
+
+
+def fg8_gather_rows(inp, n_in, row_bytes, map_, n, out, dev_status, stream=None):
+    _check(lib().fg8_gather_rows(_ptr(inp), n_in, row_bytes, _ptr(map_), n, _ptr(out),
+                                 _ptr(dev_status), _stream(stream)),
+           "fg8_gather_rows")
+
+
 def fg8_selftest_wait_timeout(which, scratch, dev_status, stream=None):
     _check(lib().fg8_selftest_wait_timeout(which, _ptr(scratch), _ptr(dev_status), _stream(stream)),
            "fg8_selftest_wait_timeout")
@@ -259,6 +297,34 @@ def quantize_act(x: torch.Tensor, topk_ids: torch.Tensor, E: int, dev_status=Non
     fg8_quantize_act(_u16(x), T, K, topk_ids, k, E, None, FG8_ROWWISE, out["xq"], out["sa"],
                      out["row_token"], out["token_row"], out["offsets"], None, None, workspace,
                      ws_bytes, st, stream)
+    out["status"] = st
+    return out
+
+
+def route_quantize_act(logits: torch.Tensor, bias: torch.Tensor, x: torch.Tensor, k: int,
+                       dev_status=None, workspace=None, stream=None):
+    """Routing (sigmoid + bias top-k) fused with permute + 1x128 quantize.
+    Returns dict(ids, affinity, xq, sa, row_token, token_row, offsets, status)."""
+    T, K = x.shape
+    E = logits.shape[1]
+    R = T * k
+    dev = x.device
+    out = dict(
+        ids=torch.empty((T, k), dtype=torch.int32, device=dev),
+        affinity=torch.empty((T, k), dtype=torch.float32, device=dev),
+        xq=torch.empty((R, K), dtype=torch.uint8, device=dev),
+        sa=torch.empty((K // 128, R), dtype=torch.float32, device=dev),
+        row_token=torch.empty(R, dtype=torch.int32, device=dev),
+        token_row=torch.empty(T * k, dtype=torch.int32, device=dev),
+        offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+    )
+    ws_bytes = fg8_quantize_act_workspace(T, k, E)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = dev_status if dev_status is not None else new_status(dev)
+    fg8_route_quantize_act(logits, bias, _u16(x), T, K, k, E, out["ids"], out["affinity"],
+                           out["xq"], out["sa"], out["row_token"], out["token_row"],
+                           out["offsets"], workspace, ws_bytes, st, stream)
     out["status"] = st
     return out
 

@@ -120,6 +120,31 @@ fg8_status fg8_quantize_act(const uint16_t* x, int64_t T, int64_t K,
                             int32_t* dev_status, fg8_stream_t stream);
 
 /*
+ * fg8_route_quantize_act -- routing fused in front of the permuting
+ * quantizer: the sigmoid-affinity top-K choice of fg8_route_topk ([DS] sec.
+ * 2.1) and the 1x128 permute + quantize of fg8_quantize_act ([K2] FP8
+ * paragraph; [DS] sec. 2.2) in one cooperative launch.  The routing phase
+ * histograms the experts it picks as it goes, so the ids are never read
+ * back for counting.  Outputs are exactly those of fg8_route_topk followed
+ * by fg8_quantize_act (permuting mode) on its ids.
+ *   logits fp32 [T][E], bias fp32 [E]      as for fg8_route_topk
+ *   x bf16 [T][K], K % 128 == 0            as for fg8_quantize_act
+ *   topk_ids int32 [T][k], affinity fp32 [T][k]   outputs (as fg8_route_topk)
+ *   xq, sa, row_token, token_row, offsets_out, workspace, ws_bytes
+ *                                          as for fg8_quantize_act
+ *   1 <= k <= min(16, E), E <= 1024.  NaN logits are outside the contract.
+ *   T == 0 only zeroes offsets_out.  The grid-wide barriers' waits are
+ *   bounded (FG8_ERR_TIMEOUT in *dev_status).
+ */
+fg8_status fg8_route_quantize_act(const float* logits, const float* bias,
+                                  const uint16_t* x, int64_t T, int64_t K, int k, int E,
+                                  int32_t* topk_ids, float* affinity,
+                                  uint8_t* xq, float* sa, int32_t* row_token,
+                                  int32_t* token_row, int32_t* offsets_out,
+                                  void* workspace, size_t ws_bytes,
+                                  int32_t* dev_status, fg8_stream_t stream);
+
+/*
  * fg8_quantize_act_noalloc -- the permuting mode of fg8_quantize_act
  * (layout FG8_ROWWISE with topk_ids) for callers that cannot allocate device
  * memory, such as a plugin whose host framework owns every allocation and
@@ -291,6 +316,9 @@ fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const float* sa,
  * fg8_quantize_act (ids) and fg8_unpermute_combine (affinity).
  *   logits fp32 [T][E]; bias fp32 [E]; ids int32 [T][k]; affinity fp32 [T][k]
  *   1 <= k <= min(16, E), E <= 1024.  NaN logits are outside the contract.
+ *   A bias of -inf masks an expert: it ranks after every finite score and,
+ *   if fewer than k experts are finite, masked experts fill the remaining
+ *   slots in ascending index order (so every row still holds k valid ids).
  */
 fg8_status fg8_route_topk(const float* logits, const float* bias, int64_t T, int E, int k,
                           int32_t* ids, float* affinity, fg8_stream_t stream);
@@ -319,6 +347,58 @@ fg8_status fg8_route_topk(const float* logits, const float* bias, int64_t T, int
 fg8_status fg8_unpermute_combine(const uint16_t* y, int64_t R, int C, const int32_t* token_row,
                                  const float* affinity, int64_t T, int k, int normalize,
                                  int out_dtype, void* out, fg8_stream_t stream);
+
+/*
+ * Expert-parallel exchange of FP8 rows (the data plane around an all-to-all;
+ * [DS] sec. 2.2: training on a cluster of NVLink / InfiniBand nodes with FP8
+ * communication, and the experts spread over the GPUs).  With W ranks, rank
+ * r owns the E_loc = E / W experts [r E_loc, (r + 1) E_loc).  After
+ * fg8_quantize_act the rows bound for rank r are the contiguous range
+ * [offsets_out[r E_loc], offsets_out[(r + 1) E_loc]) of xq, so the codes are
+ * sent as they are; these calls prepare the scales for the trip, merge what
+ * arrives into local expert order, and send expert outputs back.  The
+ * exchange itself (e.g. NCCL all-to-all) is the caller's.
+ *
+ * fg8_ep_pack_scales -- sa fp32 [K/128][R] (fg8_quantize_act's layout) ->
+ *   sa_rows fp32 [R][K/128], so the rows of each destination carry their
+ *   scales as one contiguous range too.  K % 128 == 0.
+ */
+fg8_status fg8_ep_pack_scales(const float* sa, int64_t R, int64_t K, float* sa_rows,
+                              fg8_stream_t stream);
+
+/*
+ * fg8_ep_unpack -- on the receiving rank: the W incoming segments, source 0
+ * first, each holding its rows grouped by local expert in ascending order,
+ * become the local expert order (expert-major, then source rank, then the
+ * source's own order), ready for fg8_grouped_gemm (GROUP_M).
+ *   recv_xq      E4M3 [R_recv][K] and recv_sa fp32 [R_recv][K/128]: received
+ *   counts       int32 [W][E_loc] on the device: rows source s sent for local
+ *                expert e (their sum must be R_recv)
+ *   xq, sa       E4M3 [R_recv][K], fp32 [K/128][R_recv]: local rows
+ *   offsets      int32 [E_loc + 1]: local expert e owns rows
+ *                [offsets[e], offsets[e + 1])
+ *   recv_to_local int32 [R_recv]: local row of each received row (the
+ *                combine's fg8_gather_rows map)
+ *   W * E_loc <= 2048; K % 128 == 0; xq and recv_xq 16-byte aligned.  If the
+ *   counts do not sum to R_recv, nothing is written and *dev_status gets
+ *   FG8_ERR_INVALID_ARG.
+ */
+fg8_status fg8_ep_unpack(const uint8_t* recv_xq, const float* recv_sa, const int32_t* counts,
+                         int W, int E_loc, int64_t R_recv, int64_t K, uint8_t* xq, float* sa,
+                         int32_t* offsets, int32_t* recv_to_local, int32_t* dev_status,
+                         fg8_stream_t stream);
+
+/*
+ * fg8_gather_rows -- out[i] = in[map[i]] for n rows of row_bytes bytes (a
+ * multiple of 16; in and out 16-byte aligned).  The combine side of the
+ * exchange: with map = recv_to_local, the expert outputs return to the order
+ * in which their rows arrived, so after the reverse all-to-all each rank
+ * holds its rows in its own permuted order (fg8_unpermute_combine's input).
+ * A map entry outside [0, n_in) leaves its output row untouched and writes
+ * FG8_ERR_INVALID_ARG to *dev_status.
+ */
+fg8_status fg8_gather_rows(const void* in, int64_t n_in, int64_t row_bytes, const int32_t* map,
+                           int64_t n, void* out, int32_t* dev_status, fg8_stream_t stream);
 
 /*
  * fg8_selftest_wait_timeout -- diagnostic of the failure-detection path (the

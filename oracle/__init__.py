@@ -476,3 +476,55 @@ def gemm_dense_fp64(a, sa, b, sb):
     A = dq[a] * np.repeat(sa.T.astype(np.float64), 128, axis=1)
     B = dq[b] * np.repeat(np.repeat(sb.astype(np.float64), 128, axis=0), 128, axis=1)
     return A @ B.T, np.abs(A) @ np.abs(B).T
+
+
+# --------------------------------------------------------------------------
+# expert-parallel exchange (index work, written out with plain loops)
+# --------------------------------------------------------------------------
+
+def ep_dispatch(sources, W: int):
+    """Where every routed row lands when the E experts are spread over W ranks
+    (rank r owns experts [r E/W, (r + 1) E/W)).
+
+    sources: per source rank s, (xq u8 [R_s, K], sa f32 [K/128, R_s], offsets
+    [E + 1]) of its rows grouped by expert.  Rank r receives, for each of its
+    experts in ascending order, that expert's rows from source 0, then source
+    1, ..., each source's rows in their own order.  Returns, per rank r,
+    dict(xq [n, K], sa [K/128, n], offsets [E/W + 1], origin int64 [n, 2] =
+    (source, source row) of each local row).
+    """
+    E = len(sources[0][2]) - 1
+    EL = E // W
+    K = sources[0][0].shape[1]
+    out = []
+    for r in range(W):
+        origin = []
+        offs = [0]
+        for el in range(EL):
+            e = r * EL + el
+            for s, (_, _, off) in enumerate(sources):
+                for i in range(int(off[e]), int(off[e + 1])):
+                    origin.append((s, i))
+            offs.append(len(origin))
+        n = len(origin)
+        xq = np.zeros((n, K), np.uint8)
+        sa = np.zeros((K // 128, n), np.float32)
+        for j, (s, i) in enumerate(origin):
+            xq[j] = sources[s][0][i]
+            sa[:, j] = sources[s][1][:, i]
+        out.append(dict(xq=xq, sa=sa, offsets=np.array(offs, np.int32),
+                        origin=np.array(origin, np.int64).reshape(n, 2)))
+    return out
+
+
+def ep_combine(y_locals, dispatched, rows_per_source):
+    """The reverse trip: y_locals[r] [n_r, C] are rank r's outputs of its local
+    rows (dispatched[r]["origin"] says where each came from).  Returns, per
+    source s, [rows_per_source[s], C]: each of its rows' outputs in its own
+    row order (rows that went nowhere stay zero)."""
+    C = y_locals[0].shape[1:]
+    back = [np.zeros((n,) + C, y_locals[0].dtype) for n in rows_per_source]
+    for r, d in enumerate(dispatched):
+        for j, (s, i) in enumerate(d["origin"]):
+            back[s][i] = y_locals[r][j]
+    return back

@@ -115,6 +115,17 @@ def test_next_entry_points_reject_bad_arguments_on_host(L):
     assert L.fg8_route_topk(None, 16, 4, 64, 4, 16, 16, None) == INV
     assert L.fg8_route_topk(18, 16, 4, 64, 4, 16, 16, None) == INV                     # align
     assert L.fg8_route_topk(None, None, 0, 64, 4, None, None, None) == OK
+    # fused routing + permute-quantize: k, E, K checks; null outputs; empty batch
+    assert L.fg8_route_quantize_act(16, 16, 16, 4, 256, 17, 64, 16, 16, 16, 16, 16, 16, 16, 16,
+                                    1 << 20, None, None) == INV              # k > 16
+    assert L.fg8_route_quantize_act(16, 16, 16, 4, 256, 4, 2000, 16, 16, 16, 16, 16, 16, 16, 16,
+                                    1 << 20, None, None) == INV              # E > 1024
+    assert L.fg8_route_quantize_act(16, 16, 16, 4, 200, 4, 64, 16, 16, 16, 16, 16, 16, 16, 16,
+                                    1 << 20, None, None) == INV              # K % 128
+    assert L.fg8_route_quantize_act(16, 16, 16, 4, 256, 4, 64, None, 16, 16, 16, 16, 16, 16, 16,
+                                    1 << 20, None, None) == INV              # ids null
+    assert L.fg8_route_quantize_act(16, 16, 16, 4, 256, 4, 64, 16, 16, 16, 16, 16, 16, 16, 16,
+                                    8, None, None) == INV                    # workspace small
 
 
 def test_binding_refuses_cpu_tensors(L):

@@ -74,6 +74,27 @@ def test_route_exact_ties_lower_index(oracle):
     np.testing.assert_array_equal(ids, ids_o)
 
 
+def test_route_masked_experts_minus_inf_bias(oracle):
+    """A bias of -inf masks an expert out of the ranking but it can still be
+    chosen, after every expert with a finite score, lower index first: rows
+    with fewer finite experts than k still get k distinct valid ids, equal to
+    the oracle's."""
+    rng = np.random.default_rng(95)
+    T, E, k = 300, 64, 8
+    u = rng.standard_normal((T, E)).astype(np.float32)
+    b = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    b[rng.choice(E, 60, replace=False)] = -np.inf     # only 4 finite experts
+    ids, aff = run(u, b, k)
+    ids_o, _, score = oracle.route_topk(u, b, k)
+    np.testing.assert_array_equal(np.sort(ids[:, :4], axis=1), np.sort(ids_o[:, :4], axis=1))
+    np.testing.assert_array_equal(ids[:, 4:], ids_o[:, 4:])
+    assert np.all(np.diff(np.sort(ids, axis=1), axis=1) > 0)
+    finite = np.nonzero(np.isfinite(b))[0]
+    assert np.all(np.isin(ids[:, :4], finite)) and not np.any(np.isin(ids[:, 4:], finite))
+    s = expit(np.take_along_axis(u, ids.astype(np.int64), 1).astype(np.float64))
+    assert np.all(np.abs(aff - s) <= 2.0 ** -21 * s + 1e-38)
+
+
 def test_route_dsv3_size(oracle):
     rng = np.random.default_rng(92)
     T, E, k = 8192, 256, 8
@@ -109,3 +130,35 @@ def test_route_rejects_bad_arguments():
         with pytest.raises(fg8.FG8Error) as ei:
             fg8.fg8_route_topk(u, b, 4, E, k, ids, aff)
         assert ei.value.status == fg8.FG8_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("T,E,k,K", [(8192, 256, 8, 7168), (1000, 64, 6, 256), (77, 33, 4, 384),
+                                     (300, 600, 16, 128)])
+def test_fused_route_quantize_equals_route_then_quantize(oracle, T, E, k, K):
+    """fg8_route_quantize_act (routing in the permuting kernel's histogram
+    phase) equals fg8_route_topk followed by fg8_quantize_act on its ids, bit
+    for bit; the ids pass the routing checks against the oracle and the
+    permuted codes equal the oracle's quantization of each token row."""
+    rng = np.random.default_rng(T + E + k)
+    u = rng.standard_normal((T, E)).astype(np.float32)
+    b = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    x = torch.from_numpy(rng.standard_normal((T, K)).astype(np.float32)).to(torch.bfloat16)
+    ud, bd, xd = torch.from_numpy(u).cuda(), torch.from_numpy(b).cuda(), x.cuda()
+    fused = fg8.route_quantize_act(ud, bd, xd, k)
+    ids, aff = fg8.route_topk(ud, bd, k)
+    sep = fg8.quantize_act(xd, ids, E)
+    torch.cuda.synchronize()
+    assert fused["status"].item() == 0 and sep["status"].item() == 0
+    assert torch.equal(fused["ids"], ids) and torch.equal(fused["affinity"], aff)
+    for key in ("xq", "sa", "row_token", "token_row", "offsets"):
+        assert torch.equal(fused[key], sep[key]), key
+    if T <= 1000:
+        check(oracle, u, b, k, what=f"fused T={T} E={E}")
+        ids_np = fused["ids"].cpu().numpy()
+        r = oracle.route(ids_np, E)
+        q = oracle.quantize_act(x, None, 1)
+        rt = r["row_token"]
+        assert np.array_equal(fused["offsets"].cpu().numpy(), r["offsets"])
+        assert np.array_equal(fused["row_token"].cpu().numpy(), rt)
+        assert np.array_equal(fused["xq"].cpu().numpy(), q["xq"][rt])
+        assert np.array_equal(fused["sa"].cpu().numpy(), q["sa"][:, rt])
