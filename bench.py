@@ -47,6 +47,9 @@ from fp8_fine_grained_permute_b200 import workloads as W  # noqa: E402
 
 METRIC = "grouped FP8 GEMM TFLOP/s + quantize GB/s, % of B200 FP8/HBM roofline"
 FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
+# nominal B200 figures (context next to the measured peaks): HBM3e bandwidth
+# and dense (non-sparse) FP8 tensor throughput
+NOMINAL = {"hbm_gbs": 8000.0, "fp8_tflops": 4500.0}
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -87,10 +90,26 @@ def bytes_transpose(E, N, K):
     return 2 * (E * N * K + 4 * E * N * K // 16384)
 
 
+def bytes_route_quantize(T, K, k, E):
+    """Routing fused with the permuting quantizer: the router logits in, the
+    ids and affinities out, plus the permute + quantize bytes."""
+    return 4 * T * E + 4 * E + 8 * T * k + bytes_route_quant(T, K, k, E)
+
+
 def bytes_combine(T, k, C):
     """Unpermute + combine: the k routed bf16 rows of every token in, its bf16
     row out, plus the row index and affinity of every slot."""
     return T * k * C * 2 + T * C * 2 + T * k * 8
+
+
+def nominal_of(entry: dict) -> dict:
+    """Add the fraction of the nominal peak beside the measured one."""
+    nom = NOMINAL["hbm_gbs"] if entry["unit"] == "GB/s" else NOMINAL["fp8_tflops"]
+    entry["nominal_peak"] = nom
+    entry["frac_of_nominal"] = entry["achieved"] / nom
+    if "tflops" in entry:     # an HBM-bound GEMM: its FLOP rate against the nominal FP8 peak too
+        entry["tensor_frac_of_nominal"] = entry["tflops"] / NOMINAL["fp8_tflops"]
+    return entry
 
 
 def padded_total_of(cfg: W.MoEConfig) -> int:
@@ -400,6 +419,24 @@ class Step:
                                        self.affinity, c.T, c.k, 1, self.fg8.FG8_OUT_BF16,
                                        self.comb_out, stream.cuda_stream)
 
+    def run_route_quantize(self, stream):
+        """Routing fused with the permuting quantizer (fg8_route_quantize_act)
+        on the step's X and seeded router logits."""
+        c = self.cfg
+        if not hasattr(self, "rq_ids"):
+            if not hasattr(self, "logits"):
+                self.logits = W.gen_router_logits(c, self.dev)
+                self.rbias = W.gen_expert_bias(c, self.dev)
+            e = lambda shape, dt: torch.empty(shape, dtype=dt, device=self.dev)  # noqa: E731
+            self.rq_ids, self.rq_aff = e((c.T, c.k), torch.int32), e((c.T, c.k), torch.float32)
+            self.rq_xq, self.rq_sa = e((c.R, c.hidden), torch.uint8), e((c.hidden // 128, c.R), torch.float32)
+            self.rq_rt, self.rq_tr = e(c.R, torch.int32), e(c.R, torch.int32)
+            self.rq_off = e(c.E + 1, torch.int32)
+        self.fg8.fg8_route_quantize_act(self.logits, self.rbias, self.x.view(torch.int16), c.T,
+                                        c.hidden, c.k, c.E, self.rq_ids, self.rq_aff, self.rq_xq,
+                                        self.rq_sa, self.rq_rt, self.rq_tr, self.rq_off, self.ws,
+                                        self.ws_bytes, self.status, stream.cuda_stream)
+
     def run_transpose(self, stream):
         """The standalone block transpose (fg8_transpose_blockq) of the up
         weight: the step gets WqT from the fused quantizer, this times the
@@ -654,14 +691,15 @@ class OracleBaseline:
         return {"threads": 1, "quantize_gbs": tot_b / tot_s / 1e9, "kernels": out,
                 "gemm_tflops": g / 1e12, "gemm_rows": rows}
 
-    def time_all(self, nthreads, budget_s=60.0, gemm_s=4.0, max_units=None, cache=None):
-        """`nthreads` threads over every family (budget_s / 5 seconds of timed
-        work each), then the GEMM rate on sampled rows (gemm_s seconds).
+    def time_all(self, nthreads, family_s=60.0, gemm_s=4.0, max_units=None, cache=None):
+        """`nthreads` threads over every family (at most family_s seconds of
+        timed work each: the whole workload when it fits), then the GEMM rate
+        on sampled rows (gemm_s seconds).
         max_units caps the units per family; `cache` (a dict) keeps prepared
         inputs between calls."""
         from concurrent.futures import ThreadPoolExecutor
         out, tot_b, tot_s = {}, 0.0, 0.0
-        share = budget_s / len(self.FAMILIES)
+        share = family_s
         with ThreadPoolExecutor(max_workers=nthreads) as ex:
             for fam in self.FAMILIES:
                 us = self.units(fam)
@@ -702,13 +740,13 @@ def host_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg: W.MoEConfig, source=None, budget_s: float = 60.0):
+def cpu_baseline(cfg: W.MoEConfig, source=None, family_s: float = 60.0):
     """The cpu_baseline object of the JSON line (oracle at 1 thread and at all
     usable cores; `value` is the GEMM rate at all cores)."""
     ob = OracleBaseline(cfg, source)
     n = host_threads()
     one = ob.time_1t()
-    allc = ob.time_all(n, budget_s=budget_s)
+    allc = ob.time_all(n, family_s=family_s)
     gemm_total = sum(a for b, a in work_of(cfg, padded_total_of(cfg))[0].values() if b == "tensor")
     return {
         "value": allc["gemm_tflops"], "unit": "TFLOP/s", "cores": n, "kind": "oracle",
@@ -759,7 +797,7 @@ def run_reference(args):
     res = None
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        res = ob.time_all(n, budget_s=1e9, gemm_s=1.0, max_units=n, cache=cache)
+        res = ob.time_all(n, family_s=1e9, gemm_s=1.0, max_units=n, cache=cache)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
             tf_list.append(res["gemm_tflops"])
@@ -801,7 +839,8 @@ def main():
     ap.add_argument("--config", default="dsv3", choices=sorted(W.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=60.0,
-                    help="seconds of timed oracle work for the K1-K3 families of cpu_baseline")
+                    help="cap, in seconds of timed oracle work, for each K1-K3 family of "
+                         "cpu_baseline (the whole workload is covered when it fits)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--unfused-act", action="store_true",
                     help="forward through the plain up-projection (bf16 Y) and a separately "
@@ -896,6 +935,7 @@ def main():
             q_ms += ms
         entry["share"] = ms / ms_step
         entry["traffic"] = measured_traffic(name, cfg, st.padded_total)
+        nominal_of(entry)
         kernels.append(entry)
     dom = max(kernels, key=lambda d: d["ms"])
     # K3 on its own (the step takes WqT from the fused quantizer): timed with
@@ -978,6 +1018,45 @@ def main():
                     "note": "not in the step (its ids come from the seeded host routing): "
                             "T x E fp32 logits -> top-k ids and affinities; a few MB, "
                             "L2-resident between launches, so launch- and latency-bound"})
+    # routing fused with the permute + 1x128 quantization, on its own
+    with torch.cuda.stream(stream):
+        st.run_route_quantize(stream)
+        rq0, rq1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        rq0.record(stream)
+        for _ in range(args.steps):
+            st.run_route_quantize(stream)
+        rq1.record(stream)
+    torch.cuda.synchronize()
+    rq_ms = rq0.elapsed_time(rq1) / args.steps
+    rq_bytes = bytes_route_quantize(cfg.T, cfg.hidden, cfg.k, cfg.E)
+    rq_gb = rq_bytes / (rq_ms * 1e-3) / 1e9
+    kernels.append({"kernel": "route_quantize_act", "standalone": True, "bound": "hbm",
+                    "ms": rq_ms, "achieved": rq_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": rq_gb / pk["hbm_gbs"], "share": None, "traffic": None,
+                    "replaces_ms": ro_ms + kern_ms["quant_act_permute"],
+                    "note": "not in the step (its ids come from the seeded host routing): router "
+                            "logits -> top-k ids, affinities, permuted E4M3 rows and 1x128 scales "
+                            "in one cooperative launch; replaces route_topk + quant_act_permute"})
+    # write-only HBM rate on this GPU (a fill of 8 GiB, no reads): the ceiling of
+    # kernels that mostly write, e.g. the weight gradient's fp32 output
+    fill = torch.empty(8 << 30, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        fill.fill_(1)
+        fw0, fw1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fw0.record(stream)
+        for i in range(3):
+            fill.fill_(i)
+        fw1.record(stream)
+    torch.cuda.synchronize()
+    write_gbs = 3 * fill.numel() / (fw0.elapsed_time(fw1) * 1e-3) / 1e9
+    del fill
+    for kd in kernels:
+        if kd["kernel"] == "gemm_wgrad" and kd["unit"] == "GB/s":
+            kd["write_ceiling_gbs"] = write_gbs
+            kd["frac_of_write_ceiling"] = kd["achieved"] / write_gbs
+    for kd in kernels:
+        if "nominal_peak" not in kd:
+            nominal_of(kd)
     # whole job: every rank did the same work; divide by the slowest rank's time
     gemm_ms, q_ms = all_max(pg, [gemm_ms, q_ms], dev)
     gemm_tflops = job_rate(world, gemm_flops, gemm_ms) / 1e12
@@ -1043,7 +1122,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(cfg, st, budget_s=args.cpu_budget)
+        cpu = cpu_baseline(cfg, st, family_s=args.cpu_budget)
 
     if rank == 0:
         line = {
@@ -1068,8 +1147,11 @@ def main():
                                            "step, scaled by algorithmic bytes; null if the kernel "
                                            "changed since",
                          "peak_source": f"{pk['source']}: HBM {pk['hbm_gbs']} GB/s; FP8 = "
-                                        f"{FP8_OVER_BF16} x sustained BF16 {pk['bf16_sus']} TFLOP/s"},
+                                        f"{FP8_OVER_BF16} x sustained BF16 {pk['bf16_sus']} TFLOP/s",
+                         "nominal_peak": dom["nominal_peak"], "frac_of_nominal": dom["frac_of_nominal"]},
             "kernels": kernels,
+            "hbm_write_only_gbs": {"value": write_gbs, "source": "fill of 8 GiB timed with CUDA "
+                                   "events in this run (no reads)"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clocks,

@@ -46,7 +46,10 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // are skipped).  Eight lanes own one tile (16 values each: 16-byte chunks j and
 // j + 8, so a warp's loads are whole 128-byte lines), a warp four tiles at a
 // time, two such groups (eight tiles) in flight per iteration; the tile scale
-// is computed once per 16 values.
+// is computed once per 16 values.  Neighbouring lanes then swap one 8-byte
+// half of their codes, so that each lane holds 16 consecutive codes (even
+// lane j: chunks j, j + 1; odd lane j: chunks j + 7, j + 8) and writes every
+// destination row with one aligned 16-byte store.
 __device__ __forceinline__ void quant_row(const uint16_t* __restrict__ src, int64_t K,
                                           int my_row, int nd, uint8_t* __restrict__ xq,
                                           float* __restrict__ sa, int64_t R, int lane) {
@@ -93,16 +96,25 @@ __device__ __forceinline__ void quant_row(const uint16_t* __restrict__ src, int6
                     if (q[u].exact || !fg8::bracket_agrees(c[u][x], h[u][x]))
                         c[u][x] = fg8::quant8_exact(v[u][x], q[u]);
         }
+        const bool even = (j & 1) == 0;
+        uint4 w16[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint2 give = even ? c[u][1] : c[u][0];
+            uint2 got;
+            got.x = __shfl_xor_sync(kFull, give.x, 1);
+            got.y = __shfl_xor_sync(kFull, give.y, 1);
+            w16[u] = even ? make_uint4(c[u][0].x, c[u][0].y, got.x, got.y)
+                          : make_uint4(got.x, got.y, c[u][1].x, c[u][1].y);
+        }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int tile = t0 + 4 * u + g;
-            const int64_t off = (int64_t)tile * 128 + 8 * j;
+            const int64_t off = (int64_t)tile * 128 + 8 * j + (even ? 0 : 56);
             for (int d = 0; d < nd; ++d) {
                 const int r = __shfl_sync(kFull, my_row, d);
                 if (ok[u] && r >= 0) {
-                    uint8_t* dst = xq + (int64_t)r * K + off;
-                    *reinterpret_cast<uint2*>(dst) = c[u][0];
-                    *reinterpret_cast<uint2*>(dst + 64) = c[u][1];
+                    *reinterpret_cast<uint4*>(xq + (int64_t)r * K + off) = w16[u];
                     if (j == 0) sa[(int64_t)tile * R + r] = s[u];
                 }
             }
