@@ -586,7 +586,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     nkb = v.x;
                 } else {
                     if ((tile += gridDim.x) >= total) break;
-                    nkb = decode_tile(tile, s_tiles, s_off, a, nt, e_hint).nkb;
+                    nkb = a.K / BK;   // every row-grouped tile spans the whole contraction
                 }
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(tempty_bar(buf), bphase ^ 1u, abort_flag, a.status) ||
@@ -634,6 +634,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t xphase = 0;  // gate/up epilogue: bit b = phase of buffer b's exchange barriers
         int e_hint = 0;
         bool ok = true;
+        // row-grouped mode: the scales of the next K block are loaded while this
+        // one is promoted, and during a tile's last block those of the next
+        // tile's first block, so no tile starts by waiting for a global load
+        // (two blocks ahead measured slower in the full step: it costs the
+        // promotion a spilled register)
+        float sa_n = 0.f, sb_n = 0.f;
+        bool next_loaded = false;
+        // where a row-grouped tile's scales are, for this thread
+        auto scale_ptrs = [&](const Tile& T, const float*& sap, const float*& sbp, bool& rok, bool& cok) {
+            rok = r < T.rows_valid;
+            const int c0 = T.n0 + kCols * grp;
+            cok = kSwiglu || c0 < a.N;
+            // gate/up mode: both halves cover output columns n0..n0+127; the
+            // second half's B rows (and block scales) are the up block
+            const int bcol = kSwiglu ? (grp == 0 ? T.n0 : a.N / 2 + T.n0) : c0;
+            sap = a.sa + T.rowA + r;
+            sbp = a.sb + ((int64_t)T.e * NB + bcol / 128) * KBt;
+        };
         for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
             int4 v = make_int4(0, 0, 0, 0);
             if (kGroupK) {
@@ -668,34 +686,31 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 nkb = T.nkb;
                 rows_valid = T.rows_valid;
                 out_row0 = (int)T.out_row0;
-                row_ok = r < T.rows_valid;
-                col0 = T.n0 + kCols * grp;
-                col_ok = col0 < a.N;
-                // gate/up mode: both halves cover output columns n0..n0+127; the
-                // second half's B rows (and block scales) are the up block
-                const int bcol = kSwiglu ? (grp == 0 ? T.n0 : a.N / 2 + T.n0) : col0;
-                if (kSwiglu) {
-                    col0 = T.n0;
-                    col_ok = true;
+                col0 = kSwiglu ? T.n0 : T.n0 + kCols * grp;
+                scale_ptrs(T, sa_p, sb_p, row_ok, col_ok);
+                if (!next_loaded) {
+                    sa_n = (row_ok && nkb > 0) ? __ldg(sa_p) : 0.f;
+                    sb_n = (col_ok && nkb > 0) ? __ldg(sb_p) : 0.f;
                 }
-                sa_p = a.sa + T.rowA + r;
-                sb_p = a.sb + ((int64_t)T.e * NB + bcol / 128) * KBt;
-            }
-            // row-grouped mode: the scales of the next K block are loaded while
-            // this one is promoted (two blocks ahead measured slower in the full
-            // step: it costs the promotion a spilled register)
-            float sa_n = 0.f, sb_n = 0.f;
-            if (!kGroupK) {
-                if (row_ok && nkb > 0) sa_n = __ldg(sa_p);
-                if (col_ok && nkb > 0) sb_n = __ldg(sb_p);
+                next_loaded = false;
             }
             for (int kb = 0; kb < nkb; ++kb) {
                 float s = 0.f;
                 if (!kGroupK) {
                     s = sa_n * sb_n;
                     if (kb + 1 < nkb) {
-                        if (row_ok) sa_n = __ldg(sa_p + (int64_t)(kb + 1) * a.M_total);
-                        if (col_ok) sb_n = __ldg(sb_p + kb + 1);
+                        sa_n = row_ok ? __ldg(sa_p + (int64_t)(kb + 1) * a.M_total) : 0.f;
+                        sb_n = col_ok ? __ldg(sb_p + kb + 1) : 0.f;
+                    } else if (tile + (int)gridDim.x < total) {
+                        // the next tile's first scales
+                        const Tile Tn = decode_tile(tile + (int)gridDim.x, s_tiles, s_off, a, nt, e_hint);
+                        const float* nsa;
+                        const float* nsb;
+                        bool nrok, ncok;
+                        scale_ptrs(Tn, nsa, nsb, nrok, ncok);
+                        sa_n = (nrok && Tn.nkb > 0) ? __ldg(nsa) : 0.f;
+                        sb_n = (ncok && Tn.nkb > 0) ? __ldg(nsb) : 0.f;
+                        next_loaded = true;
                     }
                 }
                 if (!mbar_wait(tfull_bar(buf), bphase, abort_flag, a.status)) {

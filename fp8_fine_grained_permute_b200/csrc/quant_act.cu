@@ -50,12 +50,14 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // half of their codes, so that each lane holds 16 consecutive codes (even
 // lane j: chunks j, j + 1; odd lane j: chunks j + 7, j + 8) and writes every
 // destination row with one aligned 16-byte store.
+// Tiles [t_lo, t_hi) of the row are done (t_lo a multiple of 8).
 __device__ __forceinline__ void quant_row(const uint16_t* __restrict__ src, int64_t K,
                                           int my_row, int nd, uint8_t* __restrict__ xq,
-                                          float* __restrict__ sa, int64_t R, int lane) {
-    const int ntile = (int)(K / 128);
+                                          float* __restrict__ sa, int64_t R, int lane,
+                                          int t_lo, int t_hi) {
+    const int ntile = t_hi;
     const int g = lane >> 3, j = lane & 7;
-    for (int t0 = 0; t0 < ntile; t0 += 8) {
+    for (int t0 = t_lo; t0 < ntile; t0 += 8) {
         uint4 v[2][2];
         bool ok[2];
 #pragma unroll
@@ -217,10 +219,18 @@ __device__ __forceinline__ void route_quant_scan_place_quantize(const RouteArgs&
     }
     __syncthreads();
 
-    // ---- phase C: quantize each token row once, store to its k rows
-    for (int64_t tok = t_begin + warp; tok < t_end; tok += kWarps) {
+    // ---- phase C: quantize each token row once, store to its k rows.  The
+    // work items are pieces of 8 tiles (1024 columns) of the chunk's token
+    // rows, dealt to the warps in turn, so that every warp gets about the same
+    // share however few tokens the chunk has.
+    const int ntile = (int)(a.K / 128);
+    const int pieces = (ntile + 7) / 8;
+    const int64_t items = (t_end - t_begin) * pieces;
+    for (int64_t it = warp; it < items; it += kWarps) {
+        const int64_t tok = t_begin + it / pieces;
+        const int pc = (int)(it % pieces);
         const int my_row = lane < k ? a.token_row[tok * k + lane] : -1;
-        quant_row(a.x + tok * a.K, a.K, my_row, k, a.xq, a.sa, R, lane);
+        quant_row(a.x + tok * a.K, a.K, my_row, k, a.xq, a.sa, R, lane, 8 * pc, min(ntile, 8 * pc + 8));
     }
 }
 
