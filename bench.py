@@ -152,27 +152,29 @@ def work_of(cfg: W.MoEConfig, padded_total: int, fused_act: bool = False):
     return w, gemm_bytes
 
 
-# DRAM bytes (read + write) per kernel family of one step, from one
-# `ncu --set full` capture of the Kanana-sized step (a few GB on the device;
-# the DeepSeek-V3-shaped step is too large to capture under full sets).  They
-# are scaled to another workload by the ratio of algorithmic bytes, and
+# DRAM bytes (read + write) per kernel family of one step: the launch list of
+# the DeepSeek-V3-shaped step (`ncu --metrics gpu__time_duration.sum,
+# dram__bytes_read.sum,dram__bytes_write.sum`, one replay pass, the bench's own
+# launches with `--steps 1 --warmup 1`; the standalone kernels' first launch).
+# They are scaled to another workload by the ratio of algorithmic bytes, and
 # dropped (traffic: null) when the kernel sources differ from the ones the
 # counters were taken on (short sha1 of the code of the kernel file and shared
 # headers, comments and whitespace removed).
 TRAFFIC_CAPTURE = {
-    "config": "kanana",
+    "config": "dsv3",
+    "fused_act": True,
     "families": {
-        "quant_act_permute": (225.1e6, "quant_act", "3d397202c14b"),
-        "quant_weight": (1023.6e6, "quant_weight", "6dd6a32fa993"),
-        "gemm_fprop_up": (680.3e6, "gemm", "5e2d6565d807"),
-        "gemm_fprop_down": (530.7e6, "gemm", "5e2d6565d807"),
-        "transpose_blockq": (345.9e6, "transpose", "3f2c2c5f91b7"),
-        "quant_act_rows": (624.1e6, "quant_act", "3d397202c14b"),
-        "gemm_dgrad": (722.0e6, "gemm", "5e2d6565d807"),
-        "quant_act_colwise": (663.7e6, "quant_act", "3d397202c14b"),
-        "gemm_wgrad": (1151.4e6, "gemm", "5e2d6565d807"),
-        "gemm_fprop_up_swiglu_quant": (479.1e6, "gemm", "5e2d6565d807"),
-        "unpermute_combine": (446.9e6, "combine", "08a271eae050"),
+        "quant_act_permute": (599.2e6, "quant_act", "6998c65ff577"),
+        "quant_weight": (41251.5e6, "quant_weight", "4f084da35b5e"),
+        "gemm_fprop_up_swiglu_quant": (8294.2e6, "gemm", "4277e7a43437"),
+        "quant_act_rows": (777.8e6, "quant_act", "6998c65ff577"),
+        "gemm_fprop_down": (4593.8e6, "gemm", "4277e7a43437"),
+        "gemm_dgrad": (8309.9e6, "gemm", "4277e7a43437"),
+        "quant_act_colwise": (1605.1e6, "quant_act", "6998c65ff577"),
+        "gemm_wgrad": (31921.1e6, "gemm", "4277e7a43437"),
+        "transpose_blockq": (14977.0e6, "transpose", "3f2c2c5f91b7"),
+        "gemm_fprop_up": (8817.3e6, "gemm", "4277e7a43437"),
+        "unpermute_combine": (1044.5e6, "combine", "08a271eae050"),
     },
 }
 # the files each family's counters depend on; fg8_common.cuh is added unless
@@ -220,7 +222,7 @@ def source_hash(group: str) -> str:
     return h.hexdigest()[:12]
 
 
-def algorithmic_bytes(family: str, cfg: W.MoEConfig, padded_total: int) -> float:
+def algorithmic_bytes(family: str, cfg: W.MoEConfig, padded_total: int, fused_act: bool = True) -> float:
     """The bytes a family must move on `cfg` (GEMMs: operands + output once)."""
     if family == "transpose_blockq":
         return bytes_transpose(cfg.E, cfg.n_up, cfg.hidden)
@@ -229,20 +231,23 @@ def algorithmic_bytes(family: str, cfg: W.MoEConfig, padded_total: int) -> float
     if family == "gemm_fprop_up_swiglu_quant":
         R, K, I = cfg.R, cfg.hidden, cfg.inter
         return R * K + cfg.E * cfg.n_up * K + R * I + 4 * R * (I // 128)
-    w, gb = work_of(cfg, padded_total)
+    w, gb = work_of(cfg, padded_total, fused_act)
     return gb.get(family, w[family][1])
 
 
-def measured_traffic(family: str, cfg: W.MoEConfig, padded_total: int):
+def measured_traffic(family: str, cfg: W.MoEConfig, padded_total: int, fused_act: bool = True):
     entry = TRAFFIC_CAPTURE["families"].get(family)
     if entry is None:
         return None
     bytes_cap, group, sha = entry
     if source_hash(group) != sha:
         return None
+    if family == "quant_act_rows" and fused_act != TRAFFIC_CAPTURE["fused_act"]:
+        return None   # the other step variant quantizes a different set of rows
     cap = W.CONFIGS[TRAFFIC_CAPTURE["config"]]
-    return bytes_cap * algorithmic_bytes(family, cfg, padded_total) / \
-        algorithmic_bytes(family, cap, padded_total_of(cap))
+    fa = TRAFFIC_CAPTURE["fused_act"]
+    return bytes_cap * algorithmic_bytes(family, cfg, padded_total, fa) / \
+        algorithmic_bytes(family, cap, padded_total_of(cap), fa)
 
 
 # --------------------------------------------------------------------------
@@ -934,7 +939,7 @@ def main():
             q_bytes += amount
             q_ms += ms
         entry["share"] = ms / ms_step
-        entry["traffic"] = measured_traffic(name, cfg, st.padded_total)
+        entry["traffic"] = measured_traffic(name, cfg, st.padded_total, st.fused_act)
         nominal_of(entry)
         kernels.append(entry)
     dom = max(kernels, key=lambda d: d["ms"])
@@ -953,7 +958,7 @@ def main():
     kernels.append({"kernel": "transpose_blockq", "standalone": True, "bound": "hbm", "ms": tr_ms,
                     "achieved": tr_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": tr_gb / pk["hbm_gbs"], "share": None,
-                    "traffic": measured_traffic("transpose_blockq", cfg, st.padded_total),
+                    "traffic": measured_traffic("transpose_blockq", cfg, st.padded_total, st.fused_act),
                     "note": "not in the step: the step's WqT comes from the fused quantizer"})
     # the up-projection kernel that the step does not use, on its own and on
     # the same operands: the plain one (bf16 Y) when the step runs the fused
@@ -974,7 +979,7 @@ def main():
         kernels.append({"kernel": alt, "standalone": True,
                         "bound": "tensor", "ms": fu_ms, "achieved": fu_tf, "peak": fp8_peak,
                         "unit": "TFLOP/s", "frac": fu_tf / fp8_peak, "share": None,
-                        "traffic": measured_traffic(alt, cfg, st.padded_total),
+                        "traffic": measured_traffic(alt, cfg, st.padded_total, st.fused_act),
                         "in_step_counterpart": in_step, "in_step_ms": kern_ms[in_step],
                         "note": "not in the step: back-to-back launches on the step's operands "
                                 "(W_up alone exceeds L2); "
@@ -997,7 +1002,7 @@ def main():
         kernels.append({"kernel": "unpermute_combine", "standalone": True, "bound": "hbm",
                         "ms": cb_ms, "achieved": cb_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
                         "frac": cb_gb / pk["hbm_gbs"], "share": None,
-                        "traffic": measured_traffic("unpermute_combine", cfg, st.padded_total),
+                        "traffic": measured_traffic("unpermute_combine", cfg, st.padded_total, st.fused_act),
                         "note": "not in the step: the layer output after the down-projection "
                                 "(T x hidden bf16 from R routed rows); back-to-back launches, "
                                 "rows larger than L2"})
@@ -1037,19 +1042,25 @@ def main():
                     "note": "not in the step (its ids come from the seeded host routing): router "
                             "logits -> top-k ids, affinities, permuted E4M3 rows and 1x128 scales "
                             "in one cooperative launch; replaces route_topk + quant_act_permute"})
-    # write-only HBM rate on this GPU (a fill of 8 GiB, no reads): the ceiling of
-    # kernels that mostly write, e.g. the weight gradient's fp32 output
+    # write-only HBM rate on this GPU (fills of 8 GiB, no reads): the ceiling of
+    # kernels that mostly write, e.g. the weight gradient's fp32 output.  torch's
+    # fill runs at a rate that depends on the element width (1-byte elements
+    # are not vectorized), so the widest view's rate is taken.
     fill = torch.empty(8 << 30, dtype=torch.uint8, device=dev)
-    with torch.cuda.stream(stream):
-        fill.fill_(1)
-        fw0, fw1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        fw0.record(stream)
-        for i in range(3):
-            fill.fill_(i)
-        fw1.record(stream)
-    torch.cuda.synchronize()
-    write_gbs = 3 * fill.numel() / (fw0.elapsed_time(fw1) * 1e-3) / 1e9
-    del fill
+    write_by_view = {}
+    for dt in (torch.uint8, torch.int32, torch.int64):
+        v = fill.view(dt)
+        with torch.cuda.stream(stream):
+            v.fill_(1)
+            fw0, fw1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fw0.record(stream)
+            for i in range(3):
+                v.fill_(i)
+            fw1.record(stream)
+        torch.cuda.synchronize()
+        write_by_view[str(dt).replace("torch.", "")] = 3 * fill.numel() / (fw0.elapsed_time(fw1) * 1e-3) / 1e9
+    write_gbs = max(write_by_view.values())
+    del fill, v
     for kd in kernels:
         if kd["kernel"] == "gemm_wgrad" and kd["unit"] == "GB/s":
             kd["write_ceiling_gbs"] = write_gbs
@@ -1142,16 +1153,17 @@ def main():
             "quantize_frac_of_hbm": quant_gbs / world / pk["hbm_gbs"],
             "roofline": {"kernel": dom["kernel"], "bound": dom["bound"], "achieved": dom["achieved"],
                          "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
-                         "traffic": measured_traffic(dom["kernel"], cfg, st.padded_total),
-                         "traffic_source": f"ncu --set full DRAM bytes of the {TRAFFIC_CAPTURE['config']} "
-                                           "step, scaled by algorithmic bytes; null if the kernel "
-                                           "changed since",
+                         "traffic": measured_traffic(dom["kernel"], cfg, st.padded_total, st.fused_act),
+                         "traffic_source": f"ncu DRAM bytes (read + write) of the {TRAFFIC_CAPTURE['config']} "
+                                           "step's launch list, scaled by algorithmic bytes; null if "
+                                           "the kernel changed since",
                          "peak_source": f"{pk['source']}: HBM {pk['hbm_gbs']} GB/s; FP8 = "
                                         f"{FP8_OVER_BF16} x sustained BF16 {pk['bf16_sus']} TFLOP/s",
                          "nominal_peak": dom["nominal_peak"], "frac_of_nominal": dom["frac_of_nominal"]},
             "kernels": kernels,
-            "hbm_write_only_gbs": {"value": write_gbs, "source": "fill of 8 GiB timed with CUDA "
-                                   "events in this run (no reads)"},
+            "hbm_write_only_gbs": {"value": write_gbs, "by_element": write_by_view,
+                                   "source": "torch fill of 8 GiB timed with CUDA events in this "
+                                   "run (no reads), fastest element width"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clocks,

@@ -88,6 +88,29 @@ FG8_DEV void tma_load_2d(const CUtensorMap* map, uint32_t dst, uint32_t bar, int
         : "memory");
 }
 
+// L2 eviction priorities for cache-hinted copies: a policy covering every
+// line the copy touches (fraction 1.0)
+FG8_DEV uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+FG8_DEV uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// tma_load_2d with an L2 eviction policy for the lines it reads
+FG8_DEV void tma_load_2d_hint(const CUtensorMap* map, uint32_t dst, uint32_t bar, int x, int y,
+                              uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0)
 FG8_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile(
@@ -102,6 +125,15 @@ FG8_DEV void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
         "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
             reinterpret_cast<uint64_t>(map)),
         "r"(src), "r"(x), "r"(y)
+        : "memory");
+}
+
+// tma_store_2d with an L2 eviction policy for the lines it writes
+FG8_DEV void tma_store_2d_hint(const CUtensorMap* map, uint32_t src, int x, int y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y), "l"(policy)
         : "memory");
 }
 

@@ -543,12 +543,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     } else {
                         mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
                     }
-                    tma_load_2d(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA);
-                    if (!kGroupK && kSwiglu) {   // B map boxes are 128 rows here
+                    if (kGroupK) {
+                        // the operands stay in L2 for the expert's other tiles
+                        // while the fp32 output streams past them (evict-first)
+                        const uint64_t keep = l2_policy_evict_last();
+                        tma_load_2d_hint(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA, keep);
+                        tma_load_2d_hint(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB,
+                                         keep);
+                    } else if (kSwiglu) {   // B map boxes are 128 rows here
+                        tma_load_2d(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA);
                         tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
                         tma_load_2d(&tmB, sA + kABytes + kBBytes / 2, full_bar(stage), T.kx0 + kb * BK,
                                     (int)T.rowB2);
                     } else {
+                        tma_load_2d(&tmA, sA, full_bar(stage), T.kx0 + kb * BK, (int)T.rowA);
                         tma_load_2d(&tmB, sA + kABytes, full_bar(stage), T.kx0 + kb * BK, (int)T.rowB);
                     }
                     if (++stage == kStages) {
@@ -572,7 +580,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
-            int e_hint = 0;
             bool ok = true;
             for (int tile = (int)blockIdx.x - (int)gridDim.x;;) {
                 int nkb;
@@ -878,6 +885,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 // warp writes its 32 rows x 128 columns as four 32 x 32 boxes,
                 // two at a time through its two 4 KB staging buffers, and
                 // TMA-stores them; the stores drain while the warp moves on.
+                // The output is written once and never read here, so its lines
+                // go first when L2 needs room.
                 // 128-byte swizzle: 16-byte chunk c of box row rr sits at chunk
                 // c ^ (rr & 7); the four lanes of a row write 32 contiguous bytes,
                 // so each 8-byte store of the warp is two conflict-free wavefronts.
@@ -906,10 +915,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         fence_async_shared();
                         __syncwarp();
                         if (lane == 0) {
+                            const uint64_t stream_out = l2_policy_evict_first();
 #pragma unroll
                             for (int bb = 0; bb < 2; ++bb)
-                                tma_store_2d(&tmOut, smem_u32(stg + bb * kBoxBytes), col0 + 64 * pr + 32 * bb,
-                                             out_row0 + 32 * quarter);
+                                tma_store_2d_hint(&tmOut, smem_u32(stg + bb * kBoxBytes), col0 + 64 * pr + 32 * bb,
+                                                  out_row0 + 32 * quarter, stream_out);
                             bulk_commit();
                         }
                         ++nbox;
