@@ -231,6 +231,9 @@ def algorithmic_bytes(family: str, cfg: W.MoEConfig, padded_total: int, fused_ac
     if family == "gemm_fprop_up_swiglu_quant":
         R, K, I = cfg.R, cfg.hidden, cfg.inter
         return R * K + cfg.E * cfg.n_up * K + R * I + 4 * R * (I // 128)
+    if family == "gemm_fprop_up":   # bf16 Y out (in the step only without the fused activation)
+        R, K, N = cfg.R, cfg.hidden, cfg.n_up
+        return R * K + cfg.E * N * K + 2 * R * N
     w, gb = work_of(cfg, padded_total, fused_act)
     return gb.get(family, w[family][1])
 
