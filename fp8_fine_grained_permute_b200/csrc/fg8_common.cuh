@@ -138,6 +138,65 @@ FG8_DEV uint2 quant8_exact(const uint4& v, const QScale& q) {
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
+// Exact codes of 8 bf16 values for a group whose fast path failed: the
+// bracket again, then an IEEE division only for the values whose brackets
+// disagree (or all of them for a subnormal scale).  Disagreement is less rare
+// than the bracket width suggests: a bf16 value divided by the scale often
+// lands exactly on a rounding midpoint between two E4M3 codes (about 5 values
+// in a thousand, 4 groups of 8 in a hundred, on normally distributed data).
+FG8_DEV uint2 quant8_redo(const uint4& v, const QScale& q) {
+    if (q.exact) return quant8_exact(v, q);
+    uint2 lo, hi;
+    quant8_bracket(v, q, lo, hi);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t& c = j < 4 ? lo.x : lo.y;
+        const uint32_t m = 0xFFu << (8 * (j & 3));
+        if (((j < 4 ? hi.x : hi.y) ^ c) & m) {
+            const float x = (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
+            c = (c & ~m) | ((cvt_e4m3x2(__fdiv_rn(x, q.s), 0.0f) & 0xFFu) << (8 * (j & 3)));
+        }
+    }
+    return lo;
+}
+
+// Warp-cooperative redo of the groups whose fast path failed.  Every lane of
+// the warp calls it with its failed groups as bits of `redo` (bit numbers
+// < 256); the warp's failed groups are listed in `list` (shared memory, `cap`
+// entries) and shared out one per lane, so the warp spends one round on them
+// however they fall on its lanes, instead of every lane redoing its own in
+// turn.  work(owner_lane, bit) redoes one group.  Returns false, having done
+// nothing, when the warp's groups do not fit the list; the caller then redoes
+// its own.
+template <class F>
+FG8_DEV bool coop_redo(uint32_t redo, uint16_t* list, int cap, F work) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t cnt = __popc(redo);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (total == 0u) return true;
+    if (total > (uint32_t)cap) return false;
+    uint32_t pos = incl - cnt;
+    while (redo != 0u) {
+        const int b = __ffs(redo) - 1;
+        redo &= redo - 1u;
+        list[pos++] = (uint16_t)((lane << 8) | b);
+    }
+    __syncwarp();
+    for (uint32_t k = lane; k < total; k += 32) {
+        const uint32_t e = list[k];
+        work((int)(e >> 8), (int)(e & 0xFFu));
+    }
+    __syncwarp();
+    return true;
+}
+
 // Quantize 8 bf16 values (one uint4) with scale context q -> 8 codes (uint2).
 FG8_DEV uint2 quant8(const uint4& v, const QScale& q) {
     uint2 lo, hi;

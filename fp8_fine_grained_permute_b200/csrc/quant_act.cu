@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, PER_LANE >= 16 ? 1 : 2) route_topk_q
 // by a 3-step shuffle, then the bracketed fast path; the tile's scale is
 // computed once per 16 values (a half-warp per tile was 8% slower).
 constexpr int kRowThreads = 256;
+constexpr int kFixCap = 64;   // failed groups a warp redoes together
 constexpr uint32_t kRowBoxBytes = 128 * 256;
 
 __global__ void __launch_bounds__(kRowThreads, 5)
@@ -313,6 +314,8 @@ quant_rows(const __grid_constant__ CUtensorMap tmX, int64_t R, int64_t K, uint8_
     extern __shared__ __align__(128) uint8_t box[];   // [128 rows][256 bytes]
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_abort;
+    __shared__ float s_sc[kRowThreads / 32][16];               // each warp's 16 row scales
+    __shared__ uint16_t s_fix[kRowThreads / 32][kFixCap];
     const int kb = blockIdx.x;
     const int64_t r0 = (int64_t)blockIdx.y * 128;
     const int t = threadIdx.x;
@@ -328,7 +331,11 @@ quant_rows(const __grid_constant__ CUtensorMap tmX, int64_t R, int64_t K, uint8_
     if (!fg8::tma::mbar_wait(bar, 0, &s_abort, status)) return;   // block-uniform in practice
     const int grp = t >> 3;        // 32 groups of 8 lanes: rows grp + 32 i
     const int l = t & 7;           // 16-byte chunks l and l + 8 of the row's tile
-#pragma unroll 2
+    // Groups whose fast path failed are only recorded here (bit 2 i + h) and
+    // redone after the loop from the staged box, so the loop stays branch-free.
+    uint32_t redo = 0;
+    const int warp = t >> 5;
+#pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int rr = grp + 32 * i;
         uint4 v[2];
@@ -338,14 +345,39 @@ quant_rows(const __grid_constant__ CUtensorMap tmX, int64_t R, int64_t K, uint8_
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
         const float sc = fg8::tile_scale(m);
-        uint2 c[2];
-        fg8::quant8xN<2>(v, fg8::make_qscale(sc), c);
+        if (l == 0) s_sc[warp][4 * i + (grp & 3)] = sc;
+        const fg8::QScale q = fg8::make_qscale(sc);
+        uint2 c[2], h[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            fg8::quant8_bracket(v[x], q, c[x], h[x]);
+            redo |= (uint32_t)(q.exact || !fg8::bracket_agrees(c[x], h[x])) << (2 * i + x);
+        }
         const int64_t r = r0 + rr;
         if (r < R) {
             uint8_t* d = xq + r * K + (int64_t)kb * 128 + l * 8;
             *reinterpret_cast<uint2*>(d) = c[0];
             *reinterpret_cast<uint2*>(d + 64) = c[1];
             if (l == 0) sa[(int64_t)kb * R + r] = sc;
+        }
+    }
+    // the exact codes of those groups over the fast-path ones, shared out over
+    // the warp (the fast-path stores were made before the warp barrier)
+    auto redo_group = [&](int owner, int b) {
+        const int to = 32 * warp + owner;
+        const int og = to >> 3, ol = to & 7, i = b >> 1, x = b & 1;
+        const int rr = og + 32 * i;
+        const int64_t r = r0 + rr;
+        const uint4 v = *reinterpret_cast<const uint4*>(box + rr * 256 + 128 * x + ol * 16);
+        const uint2 c = fg8::quant8_redo(v, fg8::make_qscale(s_sc[warp][4 * i + (og & 3)]));
+        if (r < R) *reinterpret_cast<uint2*>(xq + r * K + (int64_t)kb * 128 + ol * 8 + 64 * x) = c;
+    };
+    __syncwarp();   // the row scales
+    if (!fg8::coop_redo(redo, s_fix[warp], kFixCap, redo_group)) {
+        while (redo != 0u) {
+            const int b = __ffs(redo) - 1;
+            redo &= redo - 1u;
+            redo_group(t & 31, b);
         }
     }
 }
@@ -389,6 +421,11 @@ struct ColArgs {
 // memory with a second barrier: 4% slower.)
 constexpr uint32_t kColTileBytes = 128 * 256;
 constexpr int kColCtasPerSm = 3;
+constexpr int kColFixCap = 64;   // failed groups a warp redoes together
+// the warps' lists (from byte 0) and column-pair scales (from byte 2048) reuse s_pref
+static_assert((kColThreads / 32) * kColFixCap * 2 <= 2048 &&
+                  2048 + (kColThreads / 32) * 8 * 8 <= (kMaxE + 1) * 4,
+              "column-wise redo lists fit the tile prefix array");
 constexpr int kColGroups = 4;      // column groups per tile (grid.y)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -398,7 +435,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 
 __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColArgs a) {
     extern __shared__ __align__(128) uint8_t s_tile[];   // [2][128 rows][256 bytes]
-    __shared__ int32_t s_pref[kMaxE + 1];
+    // tiles per expert (prefix) while the CTA finds its tile; afterwards each
+    // warp's list of failed groups and its 8 column-pair scales
+    __shared__ __align__(16) int32_t s_pref[kMaxE + 1];
     __shared__ int32_t s_warp[33];
     __shared__ int32_t s_rows[128];
 
@@ -467,6 +506,8 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
     // the tokens (32 each) of pair p = 8 wp + pl
     const int wp = t >> 5, lane = t & 31;
     const int q = lane >> 3, p = 8 * wp + (lane & 7);
+    uint16_t* fix_list = reinterpret_cast<uint16_t*>(s_pref) + wp * kColFixCap;
+    float2* col_sc = reinterpret_cast<float2*>(s_pref + 512) + wp * 8;
     if (cb0 < cb1) issue(cb0, 0);
     for (int cb = cb0; cb < cb1; ++cb) {
         const int st = (cb - cb0) & 1;
@@ -478,9 +519,11 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
         uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) w[i] = src[(32 * q + i) * 64 + (p ^ (8 * q))];
-        uint32_t m = 0;
+        // column maxima as a tree (4 independent chains), not one 32-long chain
+        uint32_t mk[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+        for (int i = 0; i < 32; ++i) mk[i & 3] = __vmaxu2(mk[i & 3], w[i] & 0x7FFF7FFFu);
+        uint32_t m = __vmaxu2(__vmaxu2(mk[0], mk[1]), __vmaxu2(mk[2], mk[3]));
         m = __vmaxu2(m, __shfl_xor_sync(kFull, m, 8));
         m = __vmaxu2(m, __shfl_xor_sync(kFull, m, 16));
         const float s0 = fg8::tile_scale(__uint_as_float((m & 0xFFFFu) << 16));
@@ -494,9 +537,19 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
             v1[g] = make_uint4(__byte_perm(w[8 * g + 0], w[8 * g + 1], 0x7632), __byte_perm(w[8 * g + 2], w[8 * g + 3], 0x7632),
                                __byte_perm(w[8 * g + 4], w[8 * g + 5], 0x7632), __byte_perm(w[8 * g + 6], w[8 * g + 7], 0x7632));
         }
+        // fast-path codes of all 8 groups; the groups whose brackets disagree
+        // (bit g: column 2p, bit 4 + g: column 2p + 1) are redone exactly after
+        // the stores, so the conversions themselves stay branch-free
         uint2 c0[4], c1[4];
-        fg8::quant8xN<4>(v0, q0, c0);
-        fg8::quant8xN<4>(v1, q1, c1);
+        uint32_t redo = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            uint2 h0, h1;
+            fg8::quant8_bracket(v0[g], q0, c0[g], h0);
+            fg8::quant8_bracket(v1[g], q1, c1[g], h1);
+            redo |= (uint32_t)(q0.exact || !fg8::bracket_agrees(c0[g], h0)) << g;
+            redo |= (uint32_t)(q1.exact || !fg8::bracket_agrees(c1[g], h1)) << (4 + g);
+        }
         uint8_t* d0 = a.xqT + (col0 + 2 * p) * a.P + pcol + 32 * q;
         uint8_t* d1 = d0 + a.P;
         reinterpret_cast<uint4*>(d0)[0] = make_uint4(c0[0].x, c0[0].y, c0[1].x, c0[1].y);
@@ -505,6 +558,31 @@ __global__ void __launch_bounds__(kColThreads, kColCtasPerSm) colwise_tiles(ColA
         reinterpret_cast<uint4*>(d1)[1] = make_uint4(c1[2].x, c1[2].y, c1[3].x, c1[3].y);
         if (q == 0)
             reinterpret_cast<float2*>(a.saT + (pcol / 128) * a.C + col0)[p] = make_float2(s0, s1);
+        // exact codes of those groups from the staged words (this stage is not
+        // refilled before the next iteration's barrier) over the fast-path
+        // ones, shared out over the warp
+        if (q == 0) col_sc[lane & 7] = make_float2(s0, s1);
+        auto redo_group = [&](int owner, int b) {
+            const int oq = owner >> 3, op = 8 * wp + (owner & 7), g = b & 3, hi = b >> 2;
+            const uint32_t* wsrc = src + (32 * oq + 8 * g) * 64 + (op ^ (8 * oq));
+            uint32_t wk[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) wk[k] = wsrc[k * 64];
+            const uint32_t sel = hi ? 0x7632u : 0x5410u;
+            const uint4 v = make_uint4(__byte_perm(wk[0], wk[1], sel), __byte_perm(wk[2], wk[3], sel),
+                                       __byte_perm(wk[4], wk[5], sel), __byte_perm(wk[6], wk[7], sel));
+            const float2 sp = col_sc[owner & 7];
+            const uint2 c = fg8::quant8_redo(v, fg8::make_qscale(hi ? sp.y : sp.x));
+            *reinterpret_cast<uint2*>(a.xqT + (col0 + 2 * op + hi) * a.P + pcol + 32 * oq + 8 * g) = c;
+        };
+        if (!fg8::coop_redo(redo, fix_list, kColFixCap, redo_group)) {
+            while (redo != 0u) {
+                const int b = __ffs(redo) - 1;
+                redo &= redo - 1u;
+                redo_group(lane, b);
+            }
+            __syncwarp();
+        }
     }
 }
 

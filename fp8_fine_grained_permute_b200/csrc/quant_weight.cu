@@ -24,6 +24,7 @@ using namespace fg8::tma;
 
 constexpr int kThreads = 256;
 constexpr uint32_t kBlockBytes = 128 * 256;   // bf16 128 x 128
+constexpr int kFixCap = 64;                    // failed groups a warp redoes together
 
 // word w of code row r sits at word w ^ swz(r) of the shared code tile: conflict
 // free both for the row-wise writes and for the transposed reads below
@@ -34,12 +35,13 @@ __device__ __forceinline__ int swz(int r) { return ((r >> 2) ^ (r & 3)) & 31; }
 // the backward pass's copy costs no second read of wq.
 template <bool kT>
 __global__ void __launch_bounds__(kThreads, 5)
-quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t K,
+quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ w, int64_t N, int64_t K,
                     uint8_t* __restrict__ wq, float* __restrict__ sw, uint8_t* __restrict__ wqT,
                     float* __restrict__ swT, int32_t* status) {
     extern __shared__ __align__(128) uint8_t blk[];   // [128 rows][256 bytes]
     __shared__ __align__(8) uint64_t bar;
     __shared__ float red[kThreads / 32];
+    __shared__ uint16_t fix_list[kThreads / 32][kFixCap];
     __shared__ int abort_flag;
     const int kb = blockIdx.x, nb = blockIdx.y, e = blockIdx.z;
     const int64_t KB = K / 128, NB = N / 128;
@@ -78,16 +80,45 @@ quant_weight_blocks(const __grid_constant__ CUtensorMap tmW, int64_t N, int64_t 
     // rows per warp), so a warp barrier between the reads and the writes is
     // enough, and no second tile is needed.
     uint32_t* codes = reinterpret_cast<uint32_t*>(blk);   // row r at word 64 r
+    // Groups whose fast path failed are only recorded here (bit i) and redone
+    // after the loop, so the loop stays branch-free (a few groups in a hundred
+    // fail, mostly values that land exactly on a rounding midpoint).
+    uint32_t redo = 0;
 #pragma unroll 2
     for (int i = 0; i < 8; ++i) {
         const int r = r0 + 16 * i;
         const uint4 v = *reinterpret_cast<const uint4*>(blk + r * 256 + chunk * 16);
-        const uint2 c = fg8::quant8(v, q);
+        uint2 c, h;
+        fg8::quant8_bracket(v, q, c, h);
+        redo |= (uint32_t)(q.exact || !fg8::bracket_agrees(c, h)) << i;
         *reinterpret_cast<uint2*>(dst + (int64_t)r * K) = c;
         if (kT) {
             __syncwarp();
             codes[r * 64 + ((2 * chunk) ^ swz(r))] = c.x;
             codes[r * 64 + ((2 * chunk + 1) ^ swz(r))] = c.y;
+        }
+    }
+    // exact codes of those groups over the fast-path ones, shared out over the
+    // warp (the staged row may already hold codes, so the values come from
+    // global memory; the fast-path stores were made before the warp barrier)
+    const int warp = t >> 5;
+    auto redo_group = [&](int owner, int i) {
+        const int to = 32 * warp + owner;
+        const int ch = to & 15, r = (to >> 4) + 16 * i;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+            w + (((int64_t)e * N + (int64_t)nb * 128 + r) * K + (int64_t)kb * 128 + ch * 8)));
+        const uint2 c = fg8::quant8_redo(v, q);
+        *reinterpret_cast<uint2*>(wq + base + ch * 8 + (int64_t)r * K) = c;
+        if (kT) {
+            codes[r * 64 + ((2 * ch) ^ swz(r))] = c.x;
+            codes[r * 64 + ((2 * ch + 1) ^ swz(r))] = c.y;
+        }
+    };
+    if (!fg8::coop_redo(redo, fix_list[warp], kFixCap, redo_group)) {
+        while (redo != 0u) {
+            const int i = __ffs(redo) - 1;
+            redo &= redo - 1u;
+            redo_group(t & 31, i);
         }
     }
     const float s_out = ok ? s : __int_as_float(0x7FC00000);
@@ -139,7 +170,7 @@ fg8_status launch(const uint16_t* w, int E, int N, int K, uint8_t* wq, float* sw
         cudaSuccess)
         return FG8_ERR_CUDA;
     dim3 grid(K / 128, N / 128, E);
-    kern<<<grid, kThreads, smem, stream>>>(m, N, K, wq, sw, wqT, swT, dev_status);
+    kern<<<grid, kThreads, smem, stream>>>(m, w, N, K, wq, sw, wqT, swT, dev_status);
     return fg8h::launch_status();
 }
 
