@@ -21,6 +21,9 @@
 //    cp.async pipeline; amax per column over the tile's tokens, codes written
 //    transposed so that the token axis is contiguous (thread = 2 columns x 32
 //    tokens).
+//  quant_rows and colwise_tiles convert with the branch-free fast path and
+//  redo the groups whose bracket check failed after their main loop (per
+//  128-column block for colwise_tiles), shared out over the warp.
 #include <cuda.h>
 
 #include <mutex>

@@ -9,10 +9,11 @@
 // so each SM keeps up to five 32 KB blocks in flight without spending
 // registers on them.  The block amax is a 16-bit SIMD max over the staged
 // block, a warp shuffle and a shared-memory reduction; each thread then
-// converts 8 rows x 8 values (branch-free fast path, exact division only where
-// the bracket check asks for it) and writes them as 8-byte stores (a warp
-// writes two 128-byte code rows).  (Measured against register-resident blocks
-// of 512 threads, two per SM: 0.64 of the copy bandwidth; this one 0.97.)
+// converts 8 rows x 8 values with the branch-free fast path and writes them as
+// 8-byte stores (a warp writes two 128-byte code rows); the groups whose
+// bracket check failed are redone exactly after that loop, shared out over the
+// warp.  (Measured against register-resident blocks of 512 threads, two per
+// SM: 0.64 of the copy bandwidth; this one 0.97.)
 #include <cuda.h>
 
 #include "fg8_common.cuh"
