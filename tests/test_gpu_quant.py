@@ -400,3 +400,88 @@ def test_quantize_weight_transposed_dsv3_up_equals_separate_kernels():
     wqT2, swT2 = fg8.transpose_blockq(wq, sw)
     torch.cuda.synchronize()
     assert torch.equal(wqT, wqT2) and torch.equal(swT, swT2)
+
+
+# --------------------------------------------------------------------------
+# groups whose fast path fails: exact rounding midpoints and subnormal scales
+# --------------------------------------------------------------------------
+
+def midpoint_values(shape, seed):
+    """bf16 values that are exact midpoints between two neighbouring E4M3 codes
+    (normal and subnormal ones), random signs: with a tile maximum of 448 the
+    scale is 1 and every such value's quotient is a tie, so both brackets of
+    the fast path disagree for every value of the tile."""
+    rng = np.random.default_rng(seed)
+    j = rng.integers(0, 8, size=shape)
+    e = rng.integers(-6, 8, size=shape)                     # E4M3 normal binades below 448
+    normal = (1.0 + (2 * j + 1) / 16.0) * np.exp2(e)
+    sub = (2 * rng.integers(0, 8, size=shape) + 1) * 2.0 ** -10   # between subnormal codes
+    v = np.where(rng.random(shape) < 0.1, sub, normal)
+    v = np.where(v >= 448.0, 416.0 + 16.0, v)               # 432: the midpoint below 448
+    v *= np.where(rng.random(shape) < 0.5, -1.0, 1.0)
+    return torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
+
+
+def test_midpoint_values_are_bf16_ties():
+    v = midpoint_values((4096,), 3).float().abs().numpy()
+    assert np.all(v <= 432.0)
+    codes = np.array([float(torch.tensor(c, dtype=torch.uint8).view(torch.float8_e4m3fn).float())
+                      for c in range(0x7F)], dtype=np.float64)
+    mids = (codes[:-1] + codes[1:]) / 2
+    assert np.isin(v, mids).all()
+
+
+def test_quantize_rows_all_ties_and_subnormal_scales(oracle):
+    """Row tiles whose every value needs the exact path (ties at scale 1, and
+    tiles with a subnormal scale): more failed groups per warp than its
+    shared redo list holds."""
+    x = midpoint_values((256, 512), 21)
+    x[:, ::128] = 448.0                                     # every tile's maximum
+    x[192:, :] = torch.from_numpy(np.full((64, 512), 3, np.int16)).view(torch.bfloat16)
+    x[192:, 5] = torch.tensor(0x8007 - 0x10000, dtype=torch.int16).view(torch.bfloat16)   # -subnormal
+    xq, sa = fg8.quantize_act_rows(x.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.quantize_act(u16(x), None, 1)
+    assert np.array_equal(xq.cpu().numpy(), ref["xq"])
+    assert np.array_equal(sa.cpu().numpy(), ref["sa"])
+
+
+def test_colwise_all_ties_and_subnormal_scales(oracle):
+    counts = np.array([200, 300, 140])
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R, C = int(offsets[-1]), 384
+    y = midpoint_values((R, C), 22)
+    for e in range(2):                                      # experts 0, 1: ties at scale 1
+        for t0 in range(int(offsets[e]), int(offsets[e + 1]), 128):
+            y[t0, :] = 448.0
+    tiny = np.full((int(counts[2]), C), 2, np.int16)        # expert 2: bf16 subnormals
+    tiny[::7] = 0x8005 - 0x10000                            # negative subnormals
+    y[int(offsets[2]):] = torch.from_numpy(tiny).view(torch.bfloat16)
+    xqT, saT, padoff = fg8.quantize_act_colwise(y.cuda(), torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.quantize_act_colwise(y, offsets)
+    P = int(ref["padoff"][-1])
+    assert np.array_equal(padoff.cpu().numpy(), ref["padoff"])
+    assert np.array_equal(xqT.cpu().numpy()[:, :P], ref["xqT"][:, :P])
+    assert np.array_equal(saT.cpu().numpy()[:P // 128], ref["sT"][:P // 128])
+
+
+@pytest.mark.parametrize("transposed", [False, True])
+def test_quantize_weight_all_ties_and_subnormal_scales(oracle, transposed):
+    w = midpoint_values((2, 256, 384), 23)
+    w[:, ::128, ::128] = 448.0                              # every block's maximum
+    tiny = np.full((128, 128), 1, np.int16)
+    tiny[::3, ::5] = 0x8006 - 0x10000                       # negative subnormals
+    w[1, 128:, 256:] = torch.from_numpy(tiny).view(torch.bfloat16)   # subnormal scale
+    rwq, rsw = oracle.quantize_weight(w)
+    if transposed:
+        wq, sw, wqT, swT = fg8.quantize_weight_transposed(w.cuda())
+        torch.cuda.synchronize()
+        rwqT, rswT = oracle.transpose_blockq(rwq, rsw)
+        assert np.array_equal(wqT.cpu().numpy(), rwqT)
+        assert np.array_equal(swT.cpu().numpy(), rswT)
+    else:
+        wq, sw = fg8.quantize_weight(w.cuda())
+        torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy(), rwq)
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), rsw.view(np.uint32))
