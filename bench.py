@@ -427,6 +427,39 @@ class Step:
                                        self.affinity, c.T, c.k, 1, self.fg8.FG8_OUT_BF16,
                                        self.comb_out, stream.cuda_stream)
 
+    def ep_data_plane(self, W_ranks: int = 8):
+        """One rank's data plane of a W-rank expert-parallel layer, emulated on
+        this GPU with the step's own rows: the E experts read as W source ranks
+        of E/W local experts each (counts from the seeded routing), so the
+        permuted rows are exactly what this rank would receive, source after
+        source.  Returns the three launches (scale repack before the send, the
+        merge into local expert order after the receive, the gather of the
+        expert outputs for the way back) with their algorithmic bytes.  The
+        all-to-all itself is not part of it."""
+        c, fg8 = self.cfg, self.fg8
+        R, K, KB, EL = c.R, c.hidden, c.hidden // 128, c.E // W_ranks
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=self.dev)  # noqa: E731
+        counts = (self.offsets[1:] - self.offsets[:-1]).to(torch.int32).view(W_ranks, EL).contiguous()
+        sa_rows = e((R, KB), torch.float32)
+        xq_l, sa_l = e((R, K), torch.uint8), e((KB, R), torch.float32)
+        off_l, r2l = e(EL + 1, torch.int32), e(R, torch.int32)
+        y_back = e((R, K), torch.bfloat16)
+        y_in = self.y_dn if self.y_dn is not None else e((R, K), torch.bfloat16)
+
+        def pack(sp):
+            fg8.fg8_ep_pack_scales(self.sa, R, K, sa_rows, sp)
+
+        def unpack(sp):
+            fg8.fg8_ep_unpack(self.xq, sa_rows, counts, W_ranks, EL, R, K, xq_l, sa_l, off_l, r2l,
+                              self.status, sp)
+
+        def gather(sp):
+            fg8.fg8_gather_rows(y_in, R, K * 2, r2l, R, y_back, self.status, sp)
+
+        return [("ep_pack_scales", pack, 8 * R * KB),
+                ("ep_unpack", unpack, 2 * (R * K + 4 * R * KB) + 8 * R + 4 * (EL + 1)),
+                ("ep_gather_rows", gather, 4 * R * K + 4 * R)]
+
     def run_route_quantize(self, stream):
         """Routing fused with the permuting quantizer (fg8_route_quantize_act)
         on the step's X and seeded router logits."""
@@ -1009,6 +1042,27 @@ def main():
                         "note": "not in the step: the layer output after the down-projection "
                                 "(T x hidden bf16 from R routed rows); back-to-back launches, "
                                 "rows larger than L2"})
+    # expert-parallel data plane (one rank of 8, emulated) on its own
+    if cfg.E % 8 == 0:
+        for name, fn, nbytes in st.ep_data_plane(8):
+            with torch.cuda.stream(stream):
+                fn(stream.cuda_stream)
+                ep0, ep1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ep0.record(stream)
+                for _ in range(args.steps):
+                    fn(stream.cuda_stream)
+                ep1.record(stream)
+            torch.cuda.synchronize()
+            ep_ms = ep0.elapsed_time(ep1) / args.steps
+            ep_gb = nbytes / (ep_ms * 1e-3) / 1e9
+            kernels.append({"kernel": name, "standalone": True, "bound": "hbm", "ms": ep_ms,
+                            "achieved": ep_gb, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                            "frac": ep_gb / pk["hbm_gbs"], "share": None, "traffic": None,
+                            "note": "not in the step: one rank's data plane of an 8-rank "
+                                    "expert-parallel layer, emulated on this GPU with the step's "
+                                    "rows (the all-to-all itself is not measured: one GPU)"})
+        if st.status.item() != 0:
+            raise RuntimeError(f"expert-parallel data plane reported status {st.status.item()}")
     # sigmoid-affinity top-k routing on its own
     with torch.cuda.stream(stream):
         st.run_route(stream)
