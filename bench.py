@@ -427,6 +427,23 @@ class Step:
                                        self.affinity, c.T, c.k, 1, self.fg8.FG8_OUT_BF16,
                                        self.comb_out, stream.cuda_stream)
 
+    def run_down_combine(self, stream):
+        """The down-projection with the combine in its epilogue
+        (fg8_grouped_gemm_combine) on the step's H and W_down: -> [T, hidden]
+        fp32 token rows."""
+        c = self.cfg
+        if not hasattr(self, "dc_out"):
+            if not hasattr(self, "affinity"):
+                self.affinity = W.gen_affinity(c, self.dev)
+            self.dc_out = torch.empty((c.T, c.hidden), dtype=torch.float32, device=self.dev)
+            self.dc_ws = torch.empty(max(16, self.fg8.fg8_grouped_gemm_combine_workspace(c.R)),
+                                     dtype=torch.uint8, device=self.dev)
+        self.fg8.fg8_grouped_gemm_combine(self.hq, self.sh, self.wq_dn, self.sw_dn, self.offsets,
+                                          c.R, c.hidden, c.inter, c.E, self.row_token,
+                                          self.token_row, self.affinity, c.T, c.k, 1, self.dc_out,
+                                          self.dc_ws, self.dc_ws.numel(), self.status,
+                                          stream.cuda_stream)
+
     def ep_data_plane(self, W_ranks: int = 8):
         """One rank's data plane of a W-rank expert-parallel layer, emulated on
         this GPU with the step's own rows: the E experts read as W source ranks
@@ -1042,6 +1059,29 @@ def main():
                         "note": "not in the step: the layer output after the down-projection "
                                 "(T x hidden bf16 from R routed rows); back-to-back launches, "
                                 "rows larger than L2"})
+    # the down-projection with the combine fused into its epilogue, on its own
+    if cfg.inter:
+        with torch.cuda.stream(stream):
+            st.run_down_combine(stream)
+            dc0, dc1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            dc0.record(stream)
+            for _ in range(args.steps):
+                st.run_down_combine(stream)
+            dc1.record(stream)
+        torch.cuda.synchronize()
+        dc_ms = dc0.elapsed_time(dc1) / args.steps
+        dc_flops = 2 * cfg.R * cfg.hidden * cfg.inter
+        dc_tf = dc_flops / (dc_ms * 1e-3) / 1e12
+        kernels.append({"kernel": "gemm_fprop_down_combine", "standalone": True, "bound": "tensor",
+                        "ms": dc_ms, "achieved": dc_tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                        "frac": dc_tf / fp8_peak, "share": None, "traffic": None,
+                        "replaces_ms": kern_ms["gemm_fprop_down"] + cb_ms,
+                        "note": "not in the step: fg8_grouped_gemm_combine (the combine's "
+                                "weighted sum as fp32 reductions into the [T, hidden] output from "
+                                "the down-projection epilogue); replaces gemm_fprop_down + "
+                                "unpermute_combine"})
+        if st.status.item() != 0:
+            raise RuntimeError(f"fused down-projection + combine reported status {st.status.item()}")
     # expert-parallel data plane (one rank of 8, emulated) on its own
     if cfg.E % 8 == 0:
         for name, fn, nbytes in st.ep_data_plane(8):

@@ -174,6 +174,10 @@ struct GemmArgs {
     // 1x128 scales [I/128][M_total]
     int swiglu;
     float* out_scale;
+    // row-grouped combine mode: out = fp32 [T][N] token rows, each routed row
+    // added with its gate weight: row_tok[r], row_w[r] (fg8_grouped_gemm_combine)
+    const int32_t* row_tok;
+    const float* row_w;
 };
 
 // ---------------------------------------------------------------------------
@@ -211,6 +215,12 @@ FG8_DEV void mma_commit(uint32_t bar) {
 
 FG8_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FG8_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// out[0..3] += (x, y, z, w), one 16-byte fp32 reduction in L2 (16-byte aligned)
+FG8_DEV void red_add_v4(float* out, float x, float y, float z, float w) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(x), "f"(y), "f"(z), "f"(w)
+                 : "memory");
+}
 
 // 32 lanes x 64 consecutive fp32 columns of TMEM -> 64 registers per thread,
 // waited for inside the same asm statement (the outputs exist only after
@@ -391,7 +401,7 @@ FG8_DEV bool ring_take(TileRing& R, bool whole_warp, int4& v, volatile int* abor
 // the kernel
 // ---------------------------------------------------------------------------
 
-template <bool kGroupK, bool kSwiglu = false>
+template <bool kGroupK, bool kSwiglu = false, bool kCombine = false>
 __global__ void __launch_bounds__(Warps<kGroupK>::kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
@@ -925,6 +935,41 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         ++nbox;
                     }
                 }
+            } else if (kCombine && col_ok) {
+                // Epilogue (combine): every row times its gate weight, added
+                // into its token's row of the fp32 output with 16-byte
+                // reductions; staged like the fp32 epilogue so that each
+                // reduction instruction covers 8 rows x 64 contiguous bytes
+                uint32_t* stg = reinterpret_cast<uint32_t*>(smem + kOffStage) + ep * 32 * kStageWords;
+                uint4* my_row = reinterpret_cast<uint4*>(stg + lane * kStageWords);
+                const int sub = ((lane >> 2) & 1) * 4 + (lane >> 3);
+                const int quad = lane & 3;
+                const bool mine_ok = 32 * quarter + lane < rows_valid;
+                const int my_tok = mine_ok ? a.row_tok[out_row0 + 32 * quarter + lane] : -1;
+                const float my_w = mine_ok ? a.row_w[out_row0 + 32 * quarter + lane] : 0.f;
+                float* ob = static_cast<float*>(a.out) + col0 + 4 * quad;
+#pragma unroll
+                for (int ch = 0; ch < kCols / 16; ++ch) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        my_row[q] = make_uint4(__float_as_uint(acc[8 * ch + 2 * q].x),
+                                               __float_as_uint(acc[8 * ch + 2 * q].y),
+                                               __float_as_uint(acc[8 * ch + 2 * q + 1].x),
+                                               __float_as_uint(acc[8 * ch + 2 * q + 1].y));
+                    __syncwarp();
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int rr = 8 * g + sub;
+                        const int t = __shfl_sync(0xFFFFFFFFu, my_tok, rr);
+                        const float wgt = __shfl_sync(0xFFFFFFFFu, my_w, rr);
+                        const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStageWords + 4 * quad);
+                        if (t >= 0)
+                            red_add_v4(ob + (int64_t)t * a.N + 16 * ch, wgt * __uint_as_float(v.x),
+                                       wgt * __uint_as_float(v.y), wgt * __uint_as_float(v.z),
+                                       wgt * __uint_as_float(v.w));
+                    }
+                    __syncwarp();
+                }
             } else if (col_ok) {
             // Epilogue: 16 words of each row at a time go through this warp's
             // staging rows, then every store instruction writes 8 rows x 64
@@ -1001,6 +1046,46 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      "r"(kTmemCols)
                      : "memory");
     }
+}
+
+// Combine mode: each routed row's token and gate weight, as
+// fg8_unpermute_combine forms them (the token's kept affinities summed in
+// fp32 in slot order, one IEEE division); rows outside [0, offsets[E]) get
+// token -1.
+__global__ void combine_row_weights(const int32_t* __restrict__ offsets, int E, int64_t M_total,
+                                    const int32_t* __restrict__ row_token,
+                                    const int32_t* __restrict__ token_row,
+                                    const float* __restrict__ affinity, int64_t T, int k, int normalize,
+                                    int32_t* __restrict__ row_tok, float* __restrict__ row_w) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= M_total) return;
+    const int64_t R = offsets[E];
+    int32_t t = -1;
+    float w = 0.f;
+    if (r < R) {
+        const int32_t tt = row_token[r];
+        if (tt >= 0 && tt < T) {
+            const int32_t* tr = token_row + (int64_t)tt * k;
+            const float* af = affinity + (int64_t)tt * k;
+            float sum = 0.f, mine = 0.f;
+            bool found = false;
+            for (int j = 0; j < k; ++j) {
+                const int32_t rj = tr[j];
+                if (rj < 0 || rj >= R) continue;
+                sum = __fadd_rn(sum, af[j]);
+                if (rj == r) {
+                    mine = af[j];
+                    found = true;
+                }
+            }
+            if (found) {
+                t = tt;
+                w = !normalize ? mine : (sum == 0.f ? 0.f : __fdiv_rn(mine, sum));
+            }
+        }
+    }
+    row_tok[r] = t;
+    row_w[r] = w;
 }
 
 // ---------------------------------------------------------------------------
@@ -1094,6 +1179,8 @@ extern "C" fg8_status fg8_grouped_gemm(const uint8_t* a, const float* sa, const 
     args.ws = nullptr;
     args.swiglu = 0;
     args.out_scale = nullptr;
+    args.row_tok = nullptr;
+    args.row_w = nullptr;
     if (group_mode == FG8_GROUP_K) {
         args.ws = static_cast<unsigned int*>(workspace);
         if (cudaMemsetAsync(workspace, 0, kGroupKWorkspace, (cudaStream_t)stream) != cudaSuccess)
@@ -1151,10 +1238,87 @@ extern "C" fg8_status fg8_grouped_gemm_swiglu_quant(const uint8_t* a, const floa
     args.ws = nullptr;
     args.swiglu = 1;
     args.out_scale = sh;
+    args.row_tok = nullptr;
+    args.row_w = nullptr;
     int64_t grid = fg8h::num_sms();
     if (grid > max_tiles) grid = max_tiles;
     if (grid < 1) grid = 1;
     kern<<<(unsigned)grid, Warps<false>::kThreads, Layout<false>::kSmemBytes, (cudaStream_t)stream>>>(
         mA, mB, mA, args);
+    return fg8h::launch_status();
+}
+
+extern "C" size_t fg8_grouped_gemm_combine_workspace(int64_t M_total) {
+    return M_total > 0 ? (size_t)M_total * 8 : 0;
+}
+
+extern "C" fg8_status fg8_grouped_gemm_combine(const uint8_t* a, const float* sa, const uint8_t* b,
+                                               const float* sb, const int32_t* offsets,
+                                               int64_t M_total, int N, int K, int E,
+                                               const int32_t* row_token, const int32_t* token_row,
+                                               const float* affinity, int64_t T, int k,
+                                               int normalize, float* out, void* workspace,
+                                               size_t ws_bytes, int32_t* dev_status,
+                                               fg8_stream_t stream) {
+    if (!a || !sa || !b || !sb || !offsets || !row_token || !token_row || !affinity || !out)
+        return FG8_ERR_INVALID_ARG;
+    if (E < 1 || N < 128 || K < 128 || N % 128 || K % 128 || M_total < 0 || T < 0)
+        return FG8_ERR_INVALID_ARG;
+    if (k < 1 || k > 16) return FG8_ERR_INVALID_ARG;
+    if (E > kMaxE) return FG8_ERR_UNSUPPORTED;
+    if (!fg8h::aligned16(a) || !fg8h::aligned16(b) || !fg8h::aligned16(out) || !fg8h::aligned16(sb) ||
+        (reinterpret_cast<uintptr_t>(sa) & 3) || (reinterpret_cast<uintptr_t>(offsets) & 3) ||
+        (reinterpret_cast<uintptr_t>(row_token) & 3) || (reinterpret_cast<uintptr_t>(token_row) & 3) ||
+        (reinterpret_cast<uintptr_t>(affinity) & 3))
+        return FG8_ERR_INVALID_ARG;
+    if (M_total > INT32_MAX || T > INT32_MAX || (int64_t)E * N > INT32_MAX || T * k > INT32_MAX)
+        return FG8_ERR_UNSUPPORTED;
+    if (M_total > 0 && T > 0 &&
+        (!workspace || !fg8h::aligned16(workspace) || ws_bytes < fg8_grouped_gemm_combine_workspace(M_total)))
+        return FG8_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (T > 0 && cudaMemsetAsync(out, 0, (size_t)T * N * sizeof(float), st) != cudaSuccess)
+        return FG8_ERR_CUDA;
+    if (M_total == 0 || T == 0) return FG8_OK;
+    int32_t* row_tok = static_cast<int32_t*>(workspace);
+    float* row_w = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (size_t)M_total * 4);
+    combine_row_weights<<<(unsigned)((M_total + 255) / 256), 256, 0, st>>>(
+        offsets, E, M_total, row_token, token_row, affinity, T, k, normalize, row_tok, row_w);
+    if (cudaGetLastError() != cudaSuccess) return FG8_ERR_CUDA;
+    const int64_t nt = N / BN + (N % BN != 0);
+    const int64_t max_tiles = (M_total / BM + E) * nt;
+    if (max_tiles > INT32_MAX) return FG8_ERR_UNSUPPORTED;
+    CUtensorMap mA, mB;
+    if (!make_map(&mA, a, (uint64_t)M_total, (uint64_t)K, BM) ||
+        !make_map(&mB, b, (uint64_t)E * N, (uint64_t)K, BN))
+        return FG8_ERR_CUDA;
+    auto kern = grouped_gemm_kernel<false, false, true>;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, (const void*)kern) != cudaSuccess) return FG8_ERR_CUDA;
+    if (fa.numRegs < Warps<false>::kLaunchRegs) return FG8_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Layout<false>::kSmemBytes) != cudaSuccess)
+        return FG8_ERR_CUDA;
+    GemmArgs args;
+    args.sa = sa;
+    args.sb = sb;
+    args.offsets = offsets;
+    args.M_total = M_total;
+    args.N = N;
+    args.K = K;
+    args.E = E;
+    args.mode = FG8_GROUP_M;
+    args.out_f32 = 1;
+    args.out = out;
+    args.status = dev_status;
+    args.ws = nullptr;
+    args.swiglu = 0;
+    args.out_scale = nullptr;
+    args.row_tok = row_tok;
+    args.row_w = row_w;
+    int64_t grid = fg8h::num_sms();
+    if (grid > max_tiles) grid = max_tiles;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, Warps<false>::kThreads, Layout<false>::kSmemBytes, st>>>(mA, mB, mA, args);
     return fg8h::launch_status();
 }

@@ -93,6 +93,11 @@ def lib() -> ctypes.CDLL:
         L.fg8_route_topk.argtypes = [_P, _P, _I64, _I, _I, _P, _P, _P]
         L.fg8_unpermute_combine.restype = _I
         L.fg8_unpermute_combine.argtypes = [_P, _I64, _I, _P, _P, _I64, _I, _I, _I, _P, _P]
+        L.fg8_grouped_gemm_combine_workspace.restype = _SZ
+        L.fg8_grouped_gemm_combine_workspace.argtypes = [_I64]
+        L.fg8_grouped_gemm_combine.restype = _I
+        L.fg8_grouped_gemm_combine.argtypes = [_P, _P, _P, _P, _P, _I64, _I, _I, _I, _P, _P, _P,
+                                               _I64, _I, _I, _P, _P, _SZ, _P, _P]
         L.fg8_ep_pack_scales.restype = _I
         L.fg8_ep_pack_scales.argtypes = [_P, _I64, _I64, _P, _P]
         L.fg8_ep_unpack.restype = _I
@@ -230,6 +235,21 @@ def fg8_unpermute_combine(y, R, C, token_row, affinity, T, k, normalize, out_dty
     _check(lib().fg8_unpermute_combine(_ptr(y), R, C, _ptr(token_row), _ptr(affinity), T, k,
                                        normalize, out_dtype, _ptr(out), _stream(stream)),
            "fg8_unpermute_combine")
+
+
+def fg8_grouped_gemm_combine_workspace(M_total: int) -> int:
+    return int(lib().fg8_grouped_gemm_combine_workspace(M_total))
+
+
+def fg8_grouped_gemm_combine(a, sa, b, sb, offsets, M_total, N, K, E, row_token, token_row,
+                             affinity, T, k, normalize, out, workspace, ws_bytes, dev_status,
+                             stream=None):
+    _check(lib().fg8_grouped_gemm_combine(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(offsets),
+                                          M_total, N, K, E, _ptr(row_token), _ptr(token_row),
+                                          _ptr(affinity), T, k, normalize, _ptr(out),
+                                          _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                          _stream(stream)),
+           "fg8_grouped_gemm_combine")
 
 
 def fg8_ep_pack_scales(sa, R, K, sa_rows, stream=None):
@@ -423,6 +443,26 @@ def grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, dev_status=None, hq=None, s
     fg8_grouped_gemm_swiglu_quant(a, sa, b, sb, offsets, M_total, I, K, E, hq, sh, dev_status,
                                   stream)
     return hq, sh
+
+
+def grouped_gemm_combine(a, sa, b, sb, offsets, row_token, token_row, affinity, normalize=True,
+                         dev_status=None, out=None, stream=None, workspace=None):
+    """Row-grouped GEMM a [M,K] x b [E,N,K] with the combine in its epilogue:
+    -> out fp32 [T, N], each token's rows weighted by its gate weights."""
+    M_total, K = a.shape
+    E, N = offsets.numel() - 1, b.shape[1]
+    T, k = affinity.shape
+    dev = a.device
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(16, fg8_grouped_gemm_combine_workspace(M_total)),
+                                dtype=torch.uint8, device=dev)
+    st = dev_status if dev_status is not None else new_status(dev)
+    fg8_grouped_gemm_combine(a, sa, b, sb, offsets, M_total, N, K, E, row_token, token_row,
+                             affinity, T, k, int(bool(normalize)), out, workspace,
+                             workspace.numel(), st, stream)
+    return out
 
 
 def unpermute_combine(y, token_row, affinity, normalize=True, out_dtype=FG8_OUT_BF16, out=None,

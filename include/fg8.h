@@ -349,6 +349,38 @@ fg8_status fg8_unpermute_combine(const uint16_t* y, int64_t R, int C, const int3
                                  int out_dtype, void* out, fg8_stream_t stream);
 
 /*
+ * fg8_grouped_gemm_combine -- the down-projection and the combine in one
+ * launch: the row-grouped FP8 GEMM of fg8_grouped_gemm (FG8_GROUP_M,
+ * FG8_BSCALE_BLOCK128, the same promotion), whose epilogue multiplies every
+ * routed row by its gate weight and adds it into its token's row of the fp32
+ * output, instead of writing the rows for a separate fg8_unpermute_combine
+ * ([DS] sec. 2.1: the layer output is the affinity-weighted sum of the
+ * token's expert outputs).
+ *   out[t][c] = sum_{j < k, slot kept} w[t][j] * Y[token_row[t*k + j]][c]
+ * with Y the fp32 GEMM result (not rounded to bf16) and w[t][j] exactly as in
+ * fg8_unpermute_combine (kept affinities summed in fp32 in slot order, one
+ * IEEE division when normalize = 1).  Each product w * Y is rounded to fp32
+ * and added with an fp32 reduction in L2; the order of a token's k additions
+ * is not specified (it can differ between runs, within fp32 rounding).
+ *   a, sa, b, sb, offsets, M_total, N, K, E: as fg8_grouped_gemm, FG8_GROUP_M
+ *   row_token  int32 [M_total] (fg8_quantize_act's row_token)
+ *   token_row  int32 [T*k]; affinity fp32 [T][k]; 1 <= k <= 16
+ *   out        fp32 [T][N], zeroed by the call on the stream, then summed into
+ *   workspace  >= fg8_grouped_gemm_combine_workspace(M_total) bytes, 16-byte
+ *              aligned, caller-owned: every row's token and weight; calls that
+ *              overlap on the GPU need their own
+ * Rows with no kept slot (or outside [0, offsets[E])) add nothing; tokens
+ * with no rows get zeros.  Errors as fg8_grouped_gemm.
+ */
+size_t fg8_grouped_gemm_combine_workspace(int64_t M_total);
+fg8_status fg8_grouped_gemm_combine(const uint8_t* a, const float* sa, const uint8_t* b,
+                                    const float* sb, const int32_t* offsets, int64_t M_total,
+                                    int N, int K, int E, const int32_t* row_token,
+                                    const int32_t* token_row, const float* affinity, int64_t T,
+                                    int k, int normalize, float* out, void* workspace,
+                                    size_t ws_bytes, int32_t* dev_status, fg8_stream_t stream);
+
+/*
  * Expert-parallel exchange of FP8 rows (the data plane around an all-to-all;
  * [DS] sec. 2.2: training on a cluster of NVLink / InfiniBand nodes with FP8
  * communication, and the experts spread over the GPUs).  With W ranks, rank

@@ -284,6 +284,43 @@ def unpermute_combine(y, token_row, affinity, normalize=True):
     return out, bound
 
 
+def gemm_combine_entries(a, sa, b, sb, offsets, token_row, affinity, tokens, cols,
+                         normalize=True):
+    """The down-projection followed by the combine, at (tokens[i], cols[i]):
+        out[t][c] = sum over the token's kept slots j of w[t][j] * Y[row_j][c]
+    with Y the row-grouped product (its fp64 reference, gemm_mgrouped_entries)
+    and w the combine's gate weights (the kept affinities, normalized to sum 1
+    over the kept slots when `normalize`; a slot is kept when its row is in
+    [0, offsets[E])).  Returns (out fp64, bound fp64 = sum |w| * the GEMM's
+    |term| bound, mag fp64 = sum |w * Y|) per requested entry."""
+    offsets = np.ascontiguousarray(offsets, np.int32)
+    affinity = np.ascontiguousarray(affinity, np.float32)
+    T, k = affinity.shape
+    tr = np.ascontiguousarray(token_row, np.int32).reshape(T, k)
+    tokens = np.asarray(tokens, np.int64)
+    cols = np.asarray(cols, np.int64)
+    R = int(offsets[-1])
+    kept = (tr >= 0) & (tr < R)
+    aff = affinity.astype(np.float64)
+    sums = np.where(kept, aff, 0.0).sum(axis=1)
+    if normalize:
+        w = np.where(kept & (sums[:, None] != 0), aff / np.where(sums == 0, 1.0, sums)[:, None], 0.0)
+    else:
+        w = np.where(kept, aff, 0.0)
+    # one GEMM entry per (requested entry, kept slot)
+    ent, slot = np.nonzero(kept[tokens])
+    rows = tr[tokens[ent], slot].astype(np.int64)
+    ref, bnd = gemm_mgrouped_entries(a, sa, b, sb, offsets, rows, cols[ent])
+    wt = w[tokens[ent], slot]
+    out = np.zeros(tokens.size, np.float64)
+    bound = np.zeros(tokens.size, np.float64)
+    mag = np.zeros(tokens.size, np.float64)
+    np.add.at(out, ent, wt * ref)
+    np.add.at(bound, ent, np.abs(wt) * bnd)
+    np.add.at(mag, ent, np.abs(wt * ref))
+    return out, bound, mag
+
+
 def gemm_kgrouped_entries(a, sa, b, sb, padoff, experts, rows, cols):
     a = np.ascontiguousarray(a, np.uint8)
     sa = np.ascontiguousarray(sa, np.float32)
