@@ -164,17 +164,17 @@ TRAFFIC_CAPTURE = {
     "config": "dsv3",
     "fused_act": True,
     "families": {
-        "quant_act_permute": (599.6e6, "quant_act", "c5187dc2015d"),
-        "quant_weight": (41282.1e6, "quant_weight", "c5689f11fc37"),
-        "gemm_fprop_up_swiglu_quant": (8190.3e6, "gemm", "bccc60572796"),
-        "quant_act_rows": (778.1e6, "quant_act", "c5187dc2015d"),
-        "gemm_fprop_down": (4593.6e6, "gemm", "bccc60572796"),
-        "gemm_dgrad": (8459.3e6, "gemm", "bccc60572796"),
-        "quant_act_colwise": (1572.9e6, "quant_act", "c5187dc2015d"),
-        "gemm_wgrad": (31924.9e6, "gemm", "bccc60572796"),
-        "transpose_blockq": (14976.4e6, "transpose", "3f2c2c5f91b7"),
-        "gemm_fprop_up": (8555.6e6, "gemm", "bccc60572796"),
-        "unpermute_combine": (1044.3e6, "combine", "641810fdcb7b"),
+        "quant_act_permute": (598.5e6, "quant_act", "c5187dc2015d"),
+        "quant_weight": (41280.4e6, "quant_weight", "c5689f11fc37"),
+        "gemm_fprop_up_swiglu_quant": (7836.7e6, "gemm", "7d78004fde39"),
+        "quant_act_rows": (777.8e6, "quant_act", "c5187dc2015d"),
+        "gemm_fprop_down": (4594.1e6, "gemm", "7d78004fde39"),
+        "gemm_dgrad": (8393.9e6, "gemm", "7d78004fde39"),
+        "quant_act_colwise": (1573.4e6, "quant_act", "c5187dc2015d"),
+        "gemm_wgrad": (31920.1e6, "gemm", "7d78004fde39"),
+        "transpose_blockq": (14976.3e6, "transpose", "3f2c2c5f91b7"),
+        "gemm_fprop_up": (8460.5e6, "gemm", "7d78004fde39"),
+        "unpermute_combine": (1044.5e6, "combine", "641810fdcb7b"),
     },
 }
 # the files each family's counters depend on; fg8_common.cuh is added unless
